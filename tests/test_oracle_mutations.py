@@ -1,0 +1,124 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins
+in test_oracle_pins.py catch every one of them."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle.safe_oracle as S
+import tests.test_oracle_pins as P
+
+
+def _attention_no_scale(Q, K, V, scale, kv_len=None, q_rows=None, with_lse=False):
+    return _ORIG["attention"](Q, K, V, 1.0, kv_len, q_rows, with_lse)
+
+
+def _attention_left_padding(Q, K, V, scale, kv_len=None, q_rows=None, with_lse=False):
+    if kv_len is None:
+        return _ORIG["attention"](Q, K, V, scale, None, q_rows, with_lse)
+    M = K.shape[1]
+    Kf = np.flip(np.asarray(K, dtype=np.float64), axis=1)
+    Vf = np.flip(np.asarray(V, dtype=np.float64), axis=1)
+    return _ORIG["attention"](Q, Kf, Vf, scale, kv_len, q_rows, with_lse) if M else None
+
+
+def _attention_swapped_qk(Q, K, V, scale, kv_len=None, q_rows=None, with_lse=False):
+    # uses value rows as keys (a transposed/swapped operand)
+    return _ORIG["attention"](Q, V, V, scale, kv_len, q_rows, with_lse)
+
+
+def _softmax_no_exp(logits):
+    e = logits - np.max(logits, axis=-1, keepdims=True) + 10.0
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def _ceil_k_floor(rho_num, rho_den, N):
+    return (rho_num * N) // rho_den
+
+
+def _topk_ties_high(scores, k):
+    scores = np.asarray(scores, dtype=np.float64) + 0.0
+    B, N = scores.shape
+    Sx = np.zeros((B, k), dtype=np.int64)
+    Cx = np.zeros((B, N - k), dtype=np.int64)
+    for b in range(B):
+        order = np.lexsort((-np.arange(N), -scores[b]))
+        Sx[b] = np.sort(order[:k])
+        Cx[b] = np.sort(order[k:])
+    return Sx, Cx
+
+
+def _row_in_R_no_finite(row, dtype_code):
+    if dtype_code in (S.DTYPE_BOOL, S.DTYPE_U8):
+        return bool(np.all(row != 0))
+    return bool(np.all(row == row[0])) if row.size else True
+
+
+def _pcsp_no_mean(Q, Ky, valid_len, w, scale, heads=None):
+    H = np.asarray(Q).shape[2]
+    return _ORIG["pcsp_scores"](Q, Ky, valid_len, w, scale, heads) * H
+
+
+def _scatter_off_by_one(cache, src, Sidx, src_compact):
+    out = np.array(cache, copy=True)
+    if Sidx is None:
+        out[...] = src
+        return out
+    for b in range(out.shape[0]):
+        for r in range(Sidx.shape[1]):
+            j = min(Sidx[b, r] + 1, out.shape[1] - 1)
+            out[b, j] = src[b, r] if src_compact else src[b, Sidx[b, r]]
+    return out
+
+
+_ORIG = {n: getattr(S, n) for n in ("attention", "softmax_rows", "ceil_k", "topk_partition", "row_in_R",
+                                    "pcsp_scores", "cache_scatter")}
+
+MUTATIONS = {
+    "attention_no_scale": ("attention", _attention_no_scale),
+    "attention_left_padding": ("attention", _attention_left_padding),
+    "attention_swapped_operand": ("attention", _attention_swapped_qk),
+    "softmax_without_exp": ("softmax_rows", _softmax_no_exp),
+    "ceil_k_as_floor": ("ceil_k", _ceil_k_floor),
+    "topk_ties_to_higher_index": ("topk_partition", _topk_ties_high),
+    "classifier_ignores_nonfinite": ("row_in_R", _row_in_R_no_finite),
+    "pcsp_missing_head_mean": ("pcsp_scores", _pcsp_no_mean),
+    "scatter_off_by_one": ("cache_scatter", _scatter_off_by_one),
+}
+
+
+def _run_all_pins():
+    """Run every pin; return the number that failed."""
+    import json
+    import os
+    failures = 0
+    golden = os.path.join(os.path.dirname(P.__file__), "golden")
+    fns = [getattr(P, n) for n in dir(P) if n.startswith("test_")]
+    for fn in fns:
+        params = []
+        if fn.__name__ == "test_sdpa_closed_form_golden":
+            params = json.load(open(os.path.join(golden, "softmax_closed_form.json")))["cases"]
+        elif fn.__name__ == "test_ceil_k_golden":
+            params = json.load(open(os.path.join(golden, "topk_k_values.json")))["cases"]
+        calls = [(c,) for c in params] if params else [()]
+        for args in calls:
+            try:
+                fn(*args)
+            except Exception:  # AssertionError or a crash both count as caught
+                failures += 1
+    return failures
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    attr, bad = MUTATIONS[name]
+    monkeypatch.setattr(S, attr, bad)
+    # the package namespace re-exports the functions: patch it too
+    import oracle
+    monkeypatch.setattr(oracle, attr, bad)
+    assert _run_all_pins() > 0, f"no pin caught the planted mistake {name}"
+
+
+def test_pins_pass_unmutated():
+    assert _run_all_pins() == 0
