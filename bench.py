@@ -1,0 +1,426 @@
+"""Benchmark of the SAFE-DiT attention hot path on B200.
+
+One step = one pass of the whole hot path for one DiT block at the
+2560^2-equivalent workload (B=2, H=24, d=96, N=25600, M=128, |S|=0.25N):
+  mask classify (the all-valid [B,1,N,N] bool image mask) -> dense mask-free
+  self-attention (anchor) -> padded cross-attention -> PCSP scores + top-k ->
+  context-cache scatter -> SRSU self-attention -> SRSU cross-attention.
+Inputs (236 MB per image tensor) exceed the 126 MB L2, so no flush is needed
+between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). `value` is attention TFLOP/s of the step:
+algorithmic FLOPs of dense self-attention (4 B H N^2 d) plus SRSU
+(4 B H k N d) plus both cross-attentions (4 H d * rows * sum_b len_b) over
+the measured step time, summed over ranks (each rank runs its own replica).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mask_free_b200 import synth  # noqa: E402
+
+METRIC = "attention TFLOP/s + ms/call (dense, SRSU) at N=4096/25600; % bf16 tensor peak"
+WORKLOAD = "2560^2-equivalent SRSU step: B=2, H=24, d=96, N=25600, M=128 (len U[8,128]), k=6400 (0.25N)"
+LAUNCHES_PER_STEP = 11  # classify 3, self 1, cross 1, pcsp 3 (scores, head sum, top-k), scatter 1, srsu 1, cross(S) 1
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return {"hbm": j["hbm_gbs"], "bf16": j["bf16_tflops"], "bf16_sustained": j["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def flops(shape, lens_sum, k):
+    B, N, H, d = shape.B, shape.N, shape.H, shape.d
+    dense = 4.0 * B * H * N * N * d
+    srsu = 4.0 * B * H * k * N * d
+    cross = 4.0 * H * d * N * lens_sum
+    cross_s = 4.0 * H * d * k * lens_sum
+    return dense, srsu, cross, cross_s
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names[1:], parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def make_step_inputs(config: int, dev):
+    s = synth.CONFIGS[config]
+    g = torch.Generator(device=dev).manual_seed(1000 * config)
+
+    def bf(rows):
+        return torch.randn((s.B, rows, s.H, s.d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    lens = synth.uniform_lengths(s.B, s.len_lo, s.len_hi, synth.seed_for(config, synth.T_LEN))
+    inp = {"Q": bf(s.N), "K": bf(s.N), "V": bf(s.N), "Ky": bf(s.M), "Vy": bf(s.M),
+           "valid_len": lens.to(dev), "w": synth.content_weights(lens, s.M, synth.seed_for(config, synth.T_W)).to(dev)}
+    inp["Kc"] = (inp["K"].float() + 0.05 * torch.randn(inp["K"].shape, generator=g, device=dev)).to(torch.bfloat16)
+    inp["Vc"] = (inp["V"].float() + 0.05 * torch.randn(inp["V"].shape, generator=g, device=dev)).to(torch.bfloat16)
+    inp["mask"] = torch.ones((s.B, 1, s.N, s.N), dtype=torch.bool, device=dev)
+    return s, inp, int(lens.sum())
+
+
+class Step:
+    """One pass of the hot path; all buffers preallocated."""
+
+    def __init__(self, s, inp, dev):
+        from mask_free_b200 import ops
+        self.ops, self.s, self.inp = ops, s, inp
+        B, N, H, d, M, k = s.B, s.N, s.H, s.d, s.M, s.k
+        self.O = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+        self.Ox = torch.empty_like(self.O)
+        self.Os = torch.empty((B, k, H, d), dtype=torch.bfloat16, device=dev)
+        self.Osx = torch.empty_like(self.Os)
+        self.scores = torch.empty((B, N), dtype=torch.float32, device=dev)
+        self.S = torch.empty((B, k), dtype=torch.int32, device=dev)
+        self.C = torch.empty((B, N - k), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(ops.pcsp_workspace_bytes(B, N, H), dtype=torch.uint8, device=dev)
+        self.cls = torch.empty(3, dtype=torch.int64, device=dev)
+        self.Kc, self.Vc = inp["Kc"].clone(), inp["Vc"].clone()
+        self.events = []
+
+    def __call__(self, timed=False):
+        o, i = self.ops, self.inp
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if timed else None
+        if timed:
+            self.events.append(ev)
+        o.mask_classify(i["mask"], sync=False, result=self.cls)
+        if timed:
+            ev[0].record()
+        o.attn_self(i["Q"], i["K"], i["V"], out=self.O)
+        if timed:
+            ev[1].record()
+        o.attn_cross(i["Q"], i["Ky"], i["Vy"], i["valid_len"], out=self.Ox)
+        o.pcsp_topk(i["Q"], i["Ky"], i["valid_len"], i["w"], scores=self.scores, k=self.s.k, S=self.S, C=self.C,
+                    ws=self.ws)
+        o.ctx_cache_scatter(i["K"], i["V"], self.S, self.Kc, self.Vc, src_compact=False)
+        if timed:
+            ev[2].record()
+        o.srsu_attn(i["Q"], self.S, self.Kc, self.Vc, out=self.Os)
+        if timed:
+            ev[3].record()
+        o.attn_cross(i["Q"], i["Ky"], i["Vy"], i["valid_len"], q_idx=self.S, out=self.Osx)
+
+    def launch_times(self):
+        torch.cuda.synchronize()
+        dense = [e[0].elapsed_time(e[1]) for e in self.events]
+        srsu = [e[2].elapsed_time(e[3]) for e in self.events]
+        return dense, srsu
+
+
+def time_kernel(fn, reps=20, warm=3):
+    for _ in range(warm):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
+def kernel_table(dev, pk):
+    """ms/call and TFLOP/s of dense and SRSU at N = 4096 and 25600, the
+    memory-bound kernels' GB/s at N = 25600, and the SRSU |S|/N sweep."""
+    from mask_free_b200 import ops
+    out = {}
+    for config in (2, 4):
+        s, inp, lsum = make_step_inputs(config, dev)
+        if config == 2:
+            k = s.k
+        else:
+            k = s.k
+        S = torch.sort(torch.randperm(s.N, device=dev)[:k])[0].to(torch.int32).expand(s.B, k).contiguous()
+        O = torch.empty_like(inp["Q"])
+        Os = torch.empty((s.B, k, s.H, s.d), dtype=torch.bfloat16, device=dev)
+        dense_f, srsu_f, cross_f, _ = flops(s, lsum, k)
+        t_d = time_kernel(lambda: ops.attn_self(inp["Q"], inp["K"], inp["V"], out=O))
+        t_s = time_kernel(lambda: ops.srsu_attn(inp["Q"], S, inp["Kc"], inp["Vc"], out=Os))
+        Ox = torch.empty_like(O)
+        t_x = time_kernel(lambda: ops.attn_cross(inp["Q"], inp["Ky"], inp["Vy"], inp["valid_len"], out=Ox))
+        tag = f"N{s.N}"
+        out[f"dense_{tag}"] = {"ms": t_d, "tflops": dense_f / t_d / 1e9,
+                               "pct_bf16_burst": 100 * dense_f / t_d / 1e9 / pk["bf16"],
+                               "pct_bf16_sustained": 100 * dense_f / t_d / 1e9 / pk["bf16_sustained"]}
+        out[f"srsu_{tag}_k{k}"] = {"ms": t_s, "tflops": srsu_f / t_s / 1e9,
+                                   "pct_bf16_burst": 100 * srsu_f / t_s / 1e9 / pk["bf16"],
+                                   "pct_bf16_sustained": 100 * srsu_f / t_s / 1e9 / pk["bf16_sustained"]}
+        xbytes = 2 * 2 * s.B * s.N * s.H * s.d + 2 * 2 * s.B * s.M * s.H * s.d
+        out[f"cross_{tag}"] = {"ms": t_x, "gbs": xbytes / t_x / 1e6, "pct_hbm": 100 * xbytes / t_x / 1e6 / pk["hbm"],
+                               "tflops": cross_f / t_x / 1e9}
+        if config == 4:
+            # memory-bound kernels
+            cls = torch.empty(3, dtype=torch.int64, device=dev)
+            t_c = time_kernel(lambda: ops.mask_classify(inp["mask"], sync=False, result=cls))
+            mb = inp["mask"].numel()
+            out["classify_bool_2x1xNxN"] = {"ms": t_c, "gbs": mb / t_c / 1e6, "pct_hbm": 100 * mb / t_c / 1e6 / pk["hbm"]}
+            Kc, Vc = inp["Kc"].clone(), inp["Vc"].clone()
+            t_sc = time_kernel(lambda: ops.ctx_cache_scatter(inp["K"], inp["V"], S, Kc, Vc, src_compact=False))
+            sb = 4 * s.B * k * s.H * s.d * 2
+            out["scatter"] = {"ms": t_sc, "gbs": sb / t_sc / 1e6, "pct_hbm": 100 * sb / t_sc / 1e6 / pk["hbm"]}
+            sc = torch.empty((s.B, s.N), dtype=torch.float32, device=dev)
+            ws = torch.empty(ops.pcsp_workspace_bytes(s.B, s.N, s.H), dtype=torch.uint8, device=dev)
+            t_p = time_kernel(lambda: ops.pcsp_topk(inp["Q"], inp["Ky"], inp["valid_len"], inp["w"], scores=sc, ws=ws))
+            pb = 2 * s.B * s.N * s.H * s.d + 4 * s.B * s.H * s.N * 2 + 4 * s.B * s.N
+            out["pcsp_scores"] = {"ms": t_p, "gbs": pb / t_p / 1e6}
+            Sk = torch.empty((s.B, k), dtype=torch.int32, device=dev)
+            Ck = torch.empty((s.B, s.N - k), dtype=torch.int32, device=dev)
+            t_t = time_kernel(lambda: ops.topk_partition(sc, k, S=Sk, C=Ck))
+            out["topk"] = {"ms": t_t}
+            # SRSU wall time against |S|/N
+            sweep = {}
+            for rho in (0.1, 0.2, 0.3, 0.5, 1.0):
+                kk = max(1, math.ceil(rho * s.N))
+                Sr = torch.sort(torch.randperm(s.N, device=dev)[:kk])[0].to(torch.int32).expand(s.B, kk).contiguous()
+                Osr = torch.empty((s.B, kk, s.H, s.d), dtype=torch.bfloat16, device=dev)
+                sweep[str(rho)] = time_kernel(lambda: ops.srsu_attn(inp["Q"], Sr, inp["Kc"], inp["Vc"], out=Osr),
+                                              reps=10)
+            out["srsu_rho_sweep_ms"] = sweep
+            out["srsu_t_rho_over_t_1"] = {r: v / sweep["1.0"] for r, v in sweep.items()}
+        del inp
+        torch.cuda.empty_cache()
+    return out
+
+
+class OracleSample:
+    """The fp64 oracle (as it stands) on a bounded sample of the workload:
+    dense self-attention query rows of the N = 25600 step, all 48 (b, h)
+    pairs, against all keys."""
+
+    def __init__(self):
+        s = synth.CONFIGS[4]
+        rng = np.random.default_rng(0)
+        shape = (s.B, s.N, s.H, s.d)
+        self.s = s
+        self.Q = rng.standard_normal((s.B, 64, s.H, s.d)).astype(np.float32).astype(np.float64)
+        self.K = rng.standard_normal(shape).astype(np.float32).astype(np.float64)
+        self.V = rng.standard_normal(shape).astype(np.float32).astype(np.float64)
+
+    def run(self, budget_s):
+        import oracle as O
+        from threadpoolctl import threadpool_info
+        s = self.s
+        rows_done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < budget_s:
+            O.attention(self.Q, self.K, self.V, 1 / math.sqrt(s.d))
+            rows_done += self.Q.shape[1]
+        el = time.perf_counter() - t0
+        fl = 4.0 * s.B * s.H * rows_done * s.N * s.d
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return {"value": fl / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                "sample": f"fp64 oracle dense self-attention, {rows_done} query rows x 48 (b,h) at N=25600, "
+                          f"d=96, {el:.1f} s; {os.cpu_count()} host cores, BLAS threads {threads}",
+                "seconds": el}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    sample = OracleSample()
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals, last = [], None
+    for i in range(args.warmup + args.steps):
+        last = sample.run(budget)
+        if i >= args.warmup:
+            vals.append(last["value"])
+    v = statistics.median(vals)
+    cb = dict(last, value=v)
+    ms = None
+    print(json.dumps({
+        "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "sample": cb["sample"]},
+        "cpu_baseline": cb, "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-kernel-table", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    from mask_free_b200 import ops
+    ops.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    s, inp, lsum = make_step_inputs(4, dev)
+    step = Step(s, inp, dev)
+    f_dense, f_srsu, f_cross, f_cross_s = flops(s, lsum, s.k)
+    f_step = f_dense + f_srsu + f_cross + f_cross_s
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record()
+        for _ in range(args.steps):
+            step(timed=True)
+        t1.record()
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms_total = t0.elapsed_time(t1)
+    if dist is not None:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    value = world * f_step / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, the step, D2H of its outputs
+    host = {n: inp[n].cpu().pin_memory() for n in ("Q", "K", "V", "Ky", "Vy", "valid_len", "w")}
+    outs = [step.O, step.Ox, step.Os, step.Osx, step.S]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(2, min(args.steps, 5))
+    e0.record()
+    for _ in range(e_steps):
+        for n, t in host.items():
+            inp[n].copy_(t, non_blocking=True)
+        step()
+        for o, ho in zip(outs, host_out):
+            ho.copy_(o, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / e_steps
+    if dist is not None:
+        tt = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    e2e = {"value": world * f_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    dense_list, srsu_list = step.launch_times()
+    dense_ms = statistics.mean(dense_list)
+    achieved = f_dense / (dense_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_sustained"], "traffic": None,
+                "kernel": "flash_fwd_kernel<96> (dense self-attention)",
+                "peak_note": f"{pk['source']} sustained bf16 peak (kernel timed inside the step loop); "
+                             f"frac of burst {achieved / pk['bf16']:.3f}"}
+    kernels = {"dense_in_step_ms": dense_ms, "srsu_in_step_ms": statistics.mean(srsu_list),
+               "srsu_in_step_tflops": f_srsu / (statistics.mean(srsu_list) * 1e-3) / 1e12}
+    del step
+    torch.cuda.empty_cache()
+    if not args.no_kernel_table:
+        kernels.update(kernel_table(dev, pk))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = OracleSample().run(12.0)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs exceed L2 (236 MB per image tensor); no flush",
+                       "flops_per_step": f_step},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clk.summary(), "kernels": kernels,
+        }), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

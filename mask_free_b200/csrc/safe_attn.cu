@@ -1,0 +1,371 @@
+// safe_attn.cu - host side of the C ABI declared in include/safe_attn.h.
+//
+// One translation unit: it includes every kernel of the library, validates
+// arguments on the host, encodes the TMA tensor maps and launches on the
+// caller's stream. The library allocates no device memory.
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "safe_attn.h"
+#include "sm100.cuh"
+#include "flash_attn.cuh"
+#include "cross_attn.cuh"
+#include "aux_kernels.cuh"
+
+using namespace safe;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr float kLog2e = 1.4426950408889634f;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_d(int d) { return d == 64 || d == 96 || d == 128; }
+
+safe_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SAFE_OK : SAFE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int chunk_width(int d, int c) { return (d - 64 * c) >= 64 ? 64 : (d - 64 * c); }
+
+CUtensorMapSwizzle chunk_swizzle(int d, int c) {
+  return chunk_width(d, c) == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+}
+
+// [B, rows, H, d] bf16 tensor viewed as 4-D (d, H, rows, B); box = one
+// chunk of the head dim x 1 head x 128 rows x 1 sample. Rows past `rows`
+// read as zero.
+bool encode_rows_map(CUtensorMap* map, const void* base, int B, int rows, int H, int d, int c) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                           static_cast<cuuint64_t>(rows) * H * d * 2};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(chunk_width(d, c)), 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, chunk_swizzle(d, c), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [B*N, H*d] 2-D view for tile::gather4 (box one row high).
+bool encode_gather_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int c) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * d, static_cast<cuuint64_t>(B) * N};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(chunk_width(d, c)), 1};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, chunk_swizzle(d, c), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int nchunks(int d) { return (d + 63) / 64; }
+
+// ---------------------------------------------------------------- launches
+template <int D>
+safe_status launch_flash(FlashParams& p, cudaStream_t s) {
+  constexpr int smem = flash_smem_bytes<D>();
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(flash_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
+  dim3 grid((p.n_q + 255) / 256, p.H, p.B);
+  flash_fwd_kernel<D><<<grid, kFlashThreads, smem, s>>>(p);
+  return launch_status();
+}
+
+safe_status dispatch_flash(int d, FlashParams& p, cudaStream_t s) {
+  switch (d) {
+    case 64: return launch_flash<64>(p, s);
+    case 96: return launch_flash<96>(p, s);
+    case 128: return launch_flash<128>(p, s);
+    default: return SAFE_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D>
+safe_status launch_cross(CrossParams& p, cudaStream_t s) {
+  const int smem = cross_smem_bytes<D>(256);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [smem] {
+    attr_err = cudaFuncSetAttribute(cross_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
+  dim3 grid((p.nq + 127) / 128, p.H, p.B);
+  cross_attn_kernel<D><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
+  return launch_status();
+}
+
+safe_status dispatch_cross(int d, CrossParams& p, cudaStream_t s) {
+  switch (d) {
+    case 64: return launch_cross<64>(p, s);
+    case 96: return launch_cross<96>(p, s);
+    case 128: return launch_cross<128>(p, s);
+    default: return SAFE_ERR_UNSUPPORTED;
+  }
+}
+
+bool sizes_ok(int B, int N, int H) {
+  return B >= 1 && N >= 1 && H >= 1 && B <= 65535 && H <= 65535 &&
+         static_cast<int64_t>(B) * N <= INT_MAX;
+}
+
+// Fill the query maps of a cross-attention launch (dense or gathered rows).
+safe_status fill_cross(CrossParams& p, const void* Q, const int32_t* q_idx, int nq, const void* Ky, const void* Vy,
+                       const int32_t* valid_len, const float* w, void* O, float* partial, int B, int N, int M, int H,
+                       int d, float scale) {
+  p = CrossParams{};
+  for (int c = 0; c < nchunks(d); ++c) {
+    if (q_idx == nullptr) {
+      if (!encode_rows_map(&p.q_map[c], Q, B, N, H, d, c)) return SAFE_ERR_CUDA;
+    } else {
+      if (!encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c)) return SAFE_ERR_CUDA;
+    }
+  }
+  p.Ky = static_cast<const __nv_bfloat16*>(Ky);
+  p.Vy = static_cast<const __nv_bfloat16*>(Vy);
+  p.valid_len = valid_len;
+  p.q_idx = q_idx;
+  p.w = w;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.partial = partial;
+  p.B = B;
+  p.N = N;
+  p.M = M;
+  p.H = H;
+  p.nq = nq;
+  p.scale_log2 = scale * kLog2e;
+  p.gather = q_idx != nullptr;
+  return SAFE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int safe_abi_version(void) { return kAbiVersion; }
+
+const char* safe_status_string(int status) {
+  switch (status) {
+    case SAFE_OK: return "ok";
+    case SAFE_ERR_INVALID_ARG: return "invalid argument";
+    case SAFE_ERR_UNSUPPORTED: return "unsupported shape";
+    case SAFE_ERR_CUDA: return "CUDA error";
+    case SAFE_ERR_TIMEOUT: return "device wait timed out";
+    case SAFE_ERR_DEVICE_CHECK: return "device-side input check failed";
+    default: return "unknown status";
+  }
+}
+
+safe_status safe_mask_classify(const void* mask, int dtype, const int64_t sizes[4], const int64_t strides[4],
+                               int64_t* d_result, void* stream) {
+  if (mask == nullptr || sizes == nullptr || strides == nullptr || d_result == nullptr) return SAFE_ERR_INVALID_ARG;
+  if (dtype < SAFE_BOOL || dtype > SAFE_BF16) return SAFE_ERR_INVALID_ARG;
+  for (int a = 0; a < 4; ++a)
+    if (sizes[a] < 1 || strides[a] < 0) return SAFE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_result) & 7u) != 0) return SAFE_ERR_INVALID_ARG;
+  const int esize = (dtype <= SAFE_U8) ? 1 : (dtype == SAFE_F32 ? 4 : 2);
+  if ((reinterpret_cast<uintptr_t>(mask) % esize) != 0) return SAFE_ERR_INVALID_ARG;
+  ClassifyParams p{};
+  p.mask = static_cast<const uint8_t*>(mask);
+  p.dtype = dtype;
+  p.esize = esize;
+  p.nb = strides[0] == 0 ? 1 : sizes[0];
+  p.nh = strides[1] == 0 ? 1 : sizes[1];
+  p.nq = strides[2] == 0 ? 1 : sizes[2];
+  p.nk = strides[3] == 0 ? 1 : sizes[3];
+  p.s0 = strides[0];
+  p.s1 = strides[1];
+  p.s2 = strides[2];
+  p.s3 = strides[3];
+  p.nfail = reinterpret_cast<unsigned long long*>(d_result + 1);
+  p.first_fail = reinterpret_cast<unsigned long long*>(d_result + 2);
+  cudaStream_t s = as_stream(stream);
+  classify_init_kernel<<<1, 1, 0, s>>>(d_result);
+  const int64_t rows = p.nb * p.nh * p.nq;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (rows + 7) / 8;
+  const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 16 ? want : static_cast<int64_t>(sms) * 16);
+  classify_rows_kernel<<<grid, 256, 0, s>>>(p);
+  classify_finalize_kernel<<<1, 1, 0, s>>>(d_result);
+  return launch_status();
+}
+
+safe_status safe_mask_classify_sync(const void* mask, int dtype, const int64_t sizes[4], const int64_t strides[4],
+                                    int64_t* d_result, int64_t* h_result, void* stream) {
+  if (h_result == nullptr) return SAFE_ERR_INVALID_ARG;
+  safe_status st = safe_mask_classify(mask, dtype, sizes, strides, d_result, stream);
+  if (st != SAFE_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(h_result, d_result, 3 * sizeof(int64_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SAFE_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? SAFE_OK : SAFE_ERR_CUDA;
+}
+
+safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O, float* lse, int B, int N, int H,
+                           int d, float scale, void* stream) {
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
+  FlashParams p{};
+  for (int c = 0; c < nchunks(d); ++c) {
+    if (!encode_rows_map(&p.q_map[c], Q, B, N, H, d, c) || !encode_rows_map(&p.k_map[c], K, B, N, H, d, c) ||
+        !encode_rows_map(&p.v_map[c], V, B, N, H, d, c))
+      return SAFE_ERR_CUDA;
+  }
+  p.S = nullptr;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.n_q = N;
+  p.scale_log2 = scale * kLog2e;
+  p.gather = 0;
+  return dispatch_flash(d, p, as_stream(stream));
+}
+
+safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
+                           void* O_S, float* lse, int B, int N, int H, int d, float scale, void* stream) {
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O_S)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || k < 1 || k > N || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!q_compact && S == nullptr) return SAFE_ERR_INVALID_ARG;
+  if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
+  FlashParams p{};
+  for (int c = 0; c < nchunks(d); ++c) {
+    bool ok = encode_rows_map(&p.k_map[c], Kc, B, N, H, d, c) && encode_rows_map(&p.v_map[c], Vc, B, N, H, d, c);
+    ok = ok && (q_compact ? encode_rows_map(&p.q_map[c], Q, B, k, H, d, c)
+                          : encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c));
+    if (!ok) return SAFE_ERR_CUDA;
+  }
+  p.S = S;
+  p.O = static_cast<__nv_bfloat16*>(O_S);
+  p.lse = lse;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.n_q = k;
+  p.scale_log2 = scale * kLog2e;
+  p.gather = q_compact ? 0 : 1;
+  return dispatch_flash(d, p, as_stream(stream));
+}
+
+safe_status safe_attn_cross(const void* Q, const int32_t* q_idx, int nq, const void* Ky, const void* Vy,
+                            const int32_t* valid_len, void* O, int B, int N, int M, int H, int d, float scale,
+                            void* stream) {
+  if (!aligned16(Q) || !aligned16(Ky) || !aligned16(Vy) || !aligned16(O) || valid_len == nullptr)
+    return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || M < 1 || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (q_idx == nullptr ? nq != N : (nq < 1 || nq > N)) return SAFE_ERR_INVALID_ARG;
+  if (!supported_d(d) || M > 256) return SAFE_ERR_UNSUPPORTED;
+  CrossParams p;
+  safe_status st = fill_cross(p, Q, q_idx, nq, Ky, Vy, valid_len, nullptr, O, nullptr, B, N, M, H, d, scale);
+  if (st != SAFE_OK) return st;
+  return dispatch_cross(d, p, as_stream(stream));
+}
+
+size_t safe_pcsp_workspace_bytes(int B, int N, int H) {
+  if (B < 1 || N < 1 || H < 1) return 0;
+  return static_cast<size_t>(B) * H * N * sizeof(float);
+}
+
+safe_status safe_topk_partition(const float* scores, int B, int N, int k, int32_t* S, int32_t* C, void* stream) {
+  if (scores == nullptr || S == nullptr || B < 1 || N < 1 || k < 1 || k > N) return SAFE_ERR_INVALID_ARG;
+  topk_partition_kernel<<<B, kTopkThreads, 0, as_stream(stream)>>>(scores, N, k, S, C);
+  return launch_status();
+}
+
+safe_status safe_pcsp_topk(const void* Q, const void* Ky, const int32_t* valid_len, const float* w, int B, int N,
+                           int M, int H, int d, float scale, float* scores, int accumulate, int k, int32_t* S,
+                           int32_t* C, void* ws, size_t ws_bytes, void* stream) {
+  if (scores == nullptr || !sizes_ok(B, N, H) || k < 0 || k > N) return SAFE_ERR_INVALID_ARG;
+  if (k > 0 && S == nullptr) return SAFE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (Q != nullptr) {
+    if (!aligned16(Q) || !aligned16(Ky) || valid_len == nullptr || M < 1 || !std::isfinite(scale))
+      return SAFE_ERR_INVALID_ARG;
+    if (!supported_d(d) || M > 256) return SAFE_ERR_UNSUPPORTED;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 ||
+        ws_bytes < safe_pcsp_workspace_bytes(B, N, H))
+      return SAFE_ERR_INVALID_ARG;
+    CrossParams p;
+    // The value operand is not read when only scores are produced (O = null).
+    safe_status st = fill_cross(p, Q, nullptr, N, Ky, Ky, valid_len, w, nullptr, static_cast<float*>(ws), B, N, M,
+                                H, d, scale);
+    if (st != SAFE_OK) return st;
+    st = dispatch_cross(d, p, s);
+    if (st != SAFE_OK) return st;
+    dim3 grid((N + 255) / 256, B);
+    pcsp_reduce_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(ws), scores, B, H, N, accumulate ? 1 : 0);
+    st = launch_status();
+    if (st != SAFE_OK) return st;
+  }
+  if (k > 0) return safe_topk_partition(scores, B, N, k, S, C, stream);
+  return SAFE_OK;
+}
+
+safe_status safe_ctx_cache_scatter(const void* Ksrc, const void* Vsrc, int src_compact, const int32_t* S, int k,
+                                   void* Kc, void* Vc, int B, int N, int H, int d, void* stream) {
+  if (!aligned16(Ksrc) || !aligned16(Vsrc) || !aligned16(Kc) || !aligned16(Vc)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || d < 8 || (d % 8) != 0) return SAFE_ERR_INVALID_ARG;
+  if (S != nullptr && (k < 1 || k > N)) return SAFE_ERR_INVALID_ARG;
+  if (S == nullptr && src_compact) return SAFE_ERR_INVALID_ARG;
+  const int row_units = H * d * 2 / 16;
+  const int64_t rows = S != nullptr ? static_cast<int64_t>(B) * k : static_cast<int64_t>(B) * N;
+  const int64_t blocks = (rows * 32 + 255) / 256;
+  if (blocks > INT_MAX) return SAFE_ERR_UNSUPPORTED;
+  cache_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
+      static_cast<const uint4*>(Ksrc), static_cast<const uint4*>(Vsrc), src_compact, S, k, static_cast<uint4*>(Kc),
+      static_cast<uint4*>(Vc), B, N, row_units);
+  return launch_status();
+}
+
+safe_status safe_get_device_status(int* h_status, void* stream) {
+  if (h_status == nullptr) return SAFE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SAFE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return SAFE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return SAFE_ERR_CUDA;
+  *h_status = v;
+  return SAFE_OK;
+}
+
+safe_status safe_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return SAFE_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,255 @@
+"""Thin Python binding over libsafe_attn.so (argument marshalling only).
+
+Every function takes CUDA torch tensors, checks their dtype / shape /
+contiguity, passes raw pointers and the current torch stream to the C ABI of
+``include/safe_attn.h`` and raises ``SafeError`` on a non-OK status. All
+computation runs in the library's CUDA kernels; there is no CPU fallback: if
+the library is missing or fails to load, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsafe_attn.so")
+_lib = None
+
+SAFE_OK, SAFE_ERR_INVALID_ARG, SAFE_ERR_UNSUPPORTED, SAFE_ERR_CUDA, SAFE_ERR_TIMEOUT, SAFE_ERR_DEVICE_CHECK = range(6)
+_MASK_DTYPES = {torch.bool: 0, torch.uint8: 1, torch.float32: 2, torch.float16: 3, torch.bfloat16: 4}
+
+_vp, _i, _f, _i64p, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_int64), ctypes.c_size_t
+
+# name -> argtypes (restype is int for every entry point except the ones listed)
+_SIGS = {
+    "safe_abi_version": [],
+    "safe_mask_classify": [_vp, _i, _i64p, _i64p, _vp, _vp],
+    "safe_mask_classify_sync": [_vp, _i, _i64p, _i64p, _vp, _i64p, _vp],
+    "safe_attn_self": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp],
+    "safe_attn_cross": [_vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp],
+    "safe_pcsp_workspace_bytes": [_i, _i, _i],
+    "safe_pcsp_topk": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp],
+    "safe_topk_partition": [_vp, _i, _i, _i, _vp, _vp, _vp],
+    "safe_srsu_attn": [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp],
+    "safe_ctx_cache_scatter": [_vp, _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp],
+    "safe_get_device_status": [ctypes.POINTER(ctypes.c_int), _vp],
+    "safe_status_string": [_i],
+    "safe_selftest_wait_timeout": [ctypes.c_uint64, _vp],
+}
+_RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_status_string": ctypes.c_char_p}
+
+
+class SafeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({_status_string(status)})")
+
+
+def lib():
+    """Load libsafe_attn.so (once). Raises if it is missing: no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m mask_free_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, args in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = _RESTYPES.get(name, ctypes.c_int)
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _status_string(st: int) -> str:
+    try:
+        return lib().safe_status_string(st).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _check(fn: str, st: int):
+    if st != SAFE_OK:
+        raise SafeError(fn, st)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def abi_version() -> int:
+    return lib().safe_abi_version()
+
+
+def mask_classify(mask: torch.Tensor, sync: bool = True, result: Optional[torch.Tensor] = None):
+    """Row-constant mask classification (Eq. (6)) of a 4-D [B, H, n_q, n_k]
+    mask view (any strides; stride 0 = broadcast). Returns (verdict, nfail,
+    first_fail) as Python ints when sync, else the device int64[3] tensor."""
+    if mask.dim() != 4 or not mask.is_cuda or mask.dtype not in _MASK_DTYPES:
+        raise ValueError("mask must be a 4-D CUDA tensor of dtype bool/uint8/float32/float16/bfloat16")
+    sizes = (ctypes.c_int64 * 4)(*mask.shape)
+    strides = (ctypes.c_int64 * 4)(*mask.stride())
+    if result is None:
+        result = torch.empty(3, dtype=torch.int64, device=mask.device)
+    if sync:
+        h = (ctypes.c_int64 * 3)()
+        _check("safe_mask_classify_sync",
+               lib().safe_mask_classify_sync(_p(mask), _MASK_DTYPES[mask.dtype], sizes, strides, _p(result), h,
+                                             _stream()))
+        return int(h[0]), int(h[1]), int(h[2])
+    _check("safe_mask_classify",
+           lib().safe_mask_classify(_p(mask), _MASK_DTYPES[mask.dtype], sizes, strides, _p(result), _stream()))
+    return result
+
+
+def _scale(d: int, scale: Optional[float]) -> float:
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def attn_self(Q, K, V, scale=None, return_lse=False, out=None, lse=None):
+    """Mask-free image self-attention (Eq. (3) with the mask elided)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, n, torch.bfloat16, 4)
+    B, N, H, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V must share the shape [B, N, H, d]")
+    out = torch.empty_like(Q) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    _check("safe_attn_self", lib().safe_attn_self(_p(Q), _p(K), _p(V), _p(out), _p(lse if return_lse else None),
+                                                  B, N, H, d, _scale(d, scale), _stream()))
+    return (out, lse) if return_lse else out
+
+
+def attn_cross(Q, Ky, Vy, valid_len, q_idx=None, scale=None, out=None):
+    """Image->text cross-attention with the padding kept as valid lengths
+    (Eq. (4)); with q_idx = S the row-selective form (Eq. (17))."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(Ky, "Ky", torch.bfloat16, 4)
+    _need(Vy, "Vy", torch.bfloat16, 4)
+    _need(valid_len, "valid_len", torch.int32, 1)
+    B, N, H, d = Q.shape
+    M = Ky.shape[1]
+    nq = N
+    if q_idx is not None:
+        _need(q_idx, "q_idx", torch.int32, 2)
+        nq = q_idx.shape[1]
+    out = torch.empty((B, nq, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
+    _check("safe_attn_cross", lib().safe_attn_cross(_p(Q), _p(q_idx), nq, _p(Ky), _p(Vy), _p(valid_len), _p(out),
+                                                    B, N, M, H, d, _scale(d, scale), _stream()))
+    return out
+
+
+def pcsp_workspace_bytes(B: int, N: int, H: int) -> int:
+    return int(lib().safe_pcsp_workspace_bytes(B, N, H))
+
+
+def pcsp_topk(Q, Ky, valid_len, w=None, scores=None, accumulate=False, k=0, scale=None, S=None, C=None, ws=None):
+    """PCSP scores (Eq. (10)) for one step / layer and, if k > 0, the top-k
+    partition (Eq. (12)). Returns (scores, S, C)."""
+    if Q is not None:
+        _need(Q, "Q", torch.bfloat16, 4)
+        _need(Ky, "Ky", torch.bfloat16, 4)
+        _need(valid_len, "valid_len", torch.int32, 1)
+        B, N, H, d = Q.shape
+        M = Ky.shape[1]
+        dev = Q.device
+    else:
+        _need(scores, "scores", torch.float32, 2)
+        B, N = scores.shape
+        H, d, M = 1, 64, 1
+        dev = scores.device
+    if w is not None:
+        _need(w, "w", torch.float32, 2)
+    if scores is None:
+        scores = torch.zeros((B, N), dtype=torch.float32, device=dev)
+    if k > 0:
+        S = torch.empty((B, k), dtype=torch.int32, device=dev) if S is None else S
+        C = torch.empty((B, N - k), dtype=torch.int32, device=dev) if C is None else C
+    nbytes = pcsp_workspace_bytes(B, N, H) if Q is not None else 0
+    if Q is not None and ws is None:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _check("safe_pcsp_topk", lib().safe_pcsp_topk(
+        _p(Q), _p(Ky), _p(valid_len), _p(w), B, N, M, H, d, _scale(d, scale), _p(scores), 1 if accumulate else 0, k,
+        _p(S), _p(C), _p(ws), ws.numel() if ws is not None else 0, _stream()))
+    return scores, S, C
+
+
+def topk_partition(scores, k, S=None, C=None, with_c=True):
+    """Exact tie-stable top-k split of Eq. (12) on given scores."""
+    _need(scores, "scores", torch.float32, 2)
+    B, N = scores.shape
+    S = torch.empty((B, k), dtype=torch.int32, device=scores.device) if S is None else S
+    if with_c and C is None:
+        C = torch.empty((B, N - k), dtype=torch.int32, device=scores.device)
+    _check("safe_topk_partition", lib().safe_topk_partition(_p(scores), B, N, k, _p(S), _p(C if with_c else None),
+                                                            _stream()))
+    return S, C
+
+
+def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=None, lse=None):
+    """SRSU selective self-attention (Eq. (16)): rows S of Q against all N
+    keys of the assembled global K/V."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(S, "S", torch.int32, 2)
+    _need(Kc, "Kc", torch.bfloat16, 4)
+    _need(Vc, "Vc", torch.bfloat16, 4)
+    B, N, H, d = Kc.shape
+    k = S.shape[1]
+    out = torch.empty((B, k, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, k), dtype=torch.float32, device=Q.device)
+    _check("safe_srsu_attn", lib().safe_srsu_attn(_p(Q), 1 if q_compact else 0, _p(S), k, _p(Kc), _p(Vc), _p(out),
+                                                  _p(lse if return_lse else None), B, N, H, d, _scale(d, scale),
+                                                  _stream()))
+    return (out, lse) if return_lse else out
+
+
+def ctx_cache_scatter(Ksrc, Vsrc, S, Kc, Vc, src_compact=True):
+    """In-place cache update (Eq. (14)/(16)); S=None is the anchor refresh
+    (Eq. (19))."""
+    for t, n in ((Ksrc, "Ksrc"), (Vsrc, "Vsrc"), (Kc, "Kc"), (Vc, "Vc")):
+        _need(t, n, torch.bfloat16, 4)
+    B, N, H, d = Kc.shape
+    k = 0
+    if S is not None:
+        _need(S, "S", torch.int32, 2)
+        k = S.shape[1]
+    _check("safe_ctx_cache_scatter", lib().safe_ctx_cache_scatter(
+        _p(Ksrc), _p(Vsrc), 1 if (src_compact and S is not None) else 0, _p(S), k, _p(Kc), _p(Vc), B, N, H, d,
+        _stream()))
+    return Kc, Vc
+
+
+def device_status() -> int:
+    """Read and clear the library's device status word (synchronises)."""
+    v = ctypes.c_int(0)
+    _check("safe_get_device_status", lib().safe_get_device_status(ctypes.byref(v), _stream()))
+    return v.value
+
+
+def selftest_wait_timeout(limit_ns: int = 1_000_000) -> None:
+    """Launch the bounded-wait self-test (see safe_selftest_wait_timeout)."""
+    _check("safe_selftest_wait_timeout", lib().safe_selftest_wait_timeout(int(limit_ns), _stream()))

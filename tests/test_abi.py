@@ -1,0 +1,108 @@
+"""CPU-side checks of the C ABI: the library loads, exports every entry point
+declared in include/safe_attn.h, and rejects bad arguments on the host before
+touching the GPU."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from mask_free_b200 import build as B
+from mask_free_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "safe_attn.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(safe_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return ops.lib()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in safe_attn.h but not exported"
+    nm = subprocess.run(["nm", "-D", "--defined-only", B.LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (safe_[a-z0-9_]+)", nm))
+    assert set(names) <= exported
+    # the binding knows the signature of every declared entry point
+    assert set(names) == set(ops.exported_symbols())
+
+
+def test_library_is_built_for_sm100a_only():
+    flags = " ".join(B.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.safe_abi_version() == 1
+    assert lib.safe_status_string(0) == b"ok"
+    assert lib.safe_status_string(1) == b"invalid argument"
+    assert lib.safe_status_string(99) == b"unknown status"
+
+
+def test_workspace_size(lib):
+    assert lib.safe_pcsp_workspace_bytes(2, 25600, 24) == 2 * 25600 * 24 * 4
+    assert lib.safe_pcsp_workspace_bytes(0, 10, 1) == 0
+
+
+def test_host_validation_rejects_bad_arguments_without_gpu(lib):
+    null = None
+    # null / misaligned tensors, empty sizes, unsupported head dims
+    assert lib.safe_attn_self(null, null, null, null, null, 1, 1, 1, 96, 1.0, null) == 1
+    fake = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.safe_attn_self(odd, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null) == 1
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 0, 16, 1, 96, 1.0, null) == 1
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 0, 1, 96, 1.0, null) == 1
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 80, 1.0, null) == 2
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 96, float("nan"), null) == 1
+    # SRSU: k out of range
+    assert lib.safe_srsu_attn(fake, 0, fake, 0, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null) == 1
+    assert lib.safe_srsu_attn(fake, 0, fake, 17, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null) == 1
+    # cross: M > 256 unsupported, nq must equal N without q_idx
+    assert lib.safe_attn_cross(fake, null, 16, fake, fake, fake, fake, 1, 16, 257, 1, 96, 1.0, null) == 2
+    assert lib.safe_attn_cross(fake, null, 8, fake, fake, fake, fake, 1, 16, 16, 1, 96, 1.0, null) == 1
+    # PCSP: k > N, missing / short workspace
+    assert lib.safe_pcsp_topk(fake, fake, fake, null, 1, 16, 16, 1, 96, 1.0, fake, 0, 17, fake, null, fake, 4096,
+                              null) == 1
+    assert lib.safe_pcsp_topk(fake, fake, fake, null, 1, 16, 16, 1, 96, 1.0, fake, 0, 4, fake, null, null, 0,
+                              null) == 1
+    assert lib.safe_pcsp_topk(fake, fake, fake, null, 1, 16, 16, 2, 96, 1.0, fake, 0, 4, fake, null, fake, 64,
+                              null) == 1
+    # top-k: k = 0
+    assert lib.safe_topk_partition(fake, 1, 16, 0, fake, null, null) == 1
+    # scatter: compact source needs S; k > N
+    assert lib.safe_ctx_cache_scatter(fake, fake, 1, null, 0, fake, fake, 1, 16, 1, 96, null) == 1
+    assert lib.safe_ctx_cache_scatter(fake, fake, 1, fake, 17, fake, fake, 1, 16, 1, 96, null) == 1
+    # classifier: negative stride, zero size, bad dtype
+    sizes = (ctypes.c_int64 * 4)(1, 1, 4, 4)
+    bad_sizes = (ctypes.c_int64 * 4)(1, 1, 0, 4)
+    strides = (ctypes.c_int64 * 4)(16, 16, 4, 1)
+    neg = (ctypes.c_int64 * 4)(16, 16, 4, -1)
+    assert lib.safe_mask_classify(fake, 0, sizes, neg, fake, null) == 1
+    assert lib.safe_mask_classify(fake, 0, bad_sizes, strides, fake, null) == 1
+    assert lib.safe_mask_classify(fake, 7, sizes, strides, fake, null) == 1
+    assert lib.safe_mask_classify(ctypes.c_void_p(0x10002), 2, sizes, strides, fake, null) == 1
+    # timeout self-test: limit out of range
+    assert lib.safe_selftest_wait_timeout(0, null) == 1
+    assert lib.safe_get_device_status(null, null) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros((1, 16, 1, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.attn_self(x, x, x)
