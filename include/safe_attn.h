@@ -143,6 +143,32 @@ safe_status safe_pcsp_topk(const void* Q, const void* Ky, const int32_t* valid_l
                            int32_t* C, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Allocation-free variant of safe_pcsp_topk (the paper has no counterpart:
+ * this is an interface for callers, not a step of the method).
+ *
+ * Some callers cannot allocate device memory: code hosted inside another
+ * framework that owns every device allocation and hands its plugins no
+ * workspace, and latency-critical loops whose memory plan is fixed at
+ * start-up, where a cudaMalloc would synchronise the device or fail. This
+ * entry point takes the same arguments as safe_pcsp_topk minus the workspace
+ * and allocates nothing: the per-head partial scores go to a fixed 8 MiB
+ * array inside the library (2^21 floats), which every GPU that loads the
+ * library holds until the process exits.
+ *  - Limit: B * H * N <= 2^21 (e.g. B = 2, H = 24, N <= 43690). Larger
+ *    sizes return SAFE_ERR_UNSUPPORTED before any launch.
+ *  - Set-up: the first call on a device (with that device current) looks up
+ *    the array's device address once; make that first call before any stream
+ *    capture.
+ *  - Sharing: all calls on a device share the one array and it keeps the last
+ *    call's contents (each call overwrites the part it reads, so nothing has
+ *    to be cleared). Calls that overlap on the GPU (e.g. on two streams at
+ *    once) race on it: serialise them.
+ */
+safe_status safe_pcsp_topk_noalloc(const void* Q, const void* Ky, const int32_t* valid_len, const float* w, int B,
+                                   int N, int M, int H, int d, float scale, float* scores, int accumulate, int k,
+                                   int32_t* S, int32_t* C, void* stream);
+
+/*
  * Top-k partition of Eq. (12) on given scores: S[b] = the k tokens with the
  * largest score, ordered by (score descending, index ascending) so ties go to
  * the lower index; -0.0 ranks as +0.0; C[b] = the other N-k tokens. Both are

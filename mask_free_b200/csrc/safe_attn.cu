@@ -169,6 +169,39 @@ safe_status fill_cross(CrossParams& p, const void* Q, const int32_t* q_idx, int 
 
 }  // namespace
 
+// ---------------------------------------------------------------- allocation-free PCSP
+// Scratch for safe_pcsp_topk_noalloc: the per-head partial scores [B, H, N]
+// live in this fixed array, which every GPU that loads the library keeps
+// until the process exits. Host code must not use the name as an address (it
+// is only a host-side stand-in); the device address comes from
+// cudaGetSymbolAddress, looked up once per device below.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 21;  // 2 Mi floats = 8 MiB
+static __device__ __align__(256) float g_pcsp_noalloc_scratch[kNoAllocScratchFloats];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on the
+// first call made with that device current).
+safe_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAFE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SAFE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pcsp_noalloc_scratch) != cudaSuccess || p == nullptr) return SAFE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SAFE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int safe_abi_version(void) { return kAbiVersion; }
@@ -332,6 +365,25 @@ safe_status safe_pcsp_topk(const void* Q, const void* Ky, const int32_t* valid_l
   }
   if (k > 0) return safe_topk_partition(scores, B, N, k, S, C, stream);
   return SAFE_OK;
+}
+
+safe_status safe_pcsp_topk_noalloc(const void* Q, const void* Ky, const int32_t* valid_len, const float* w, int B,
+                                   int N, int M, int H, int d, float scale, float* scores, int accumulate, int k,
+                                   int32_t* S, int32_t* C, void* stream) {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (Q != nullptr) {
+    if (B < 1 || N < 1 || H < 1) return SAFE_ERR_INVALID_ARG;
+    const size_t need = safe_pcsp_workspace_bytes(B, N, H);
+    if (need > sizeof(g_pcsp_noalloc_scratch)) return SAFE_ERR_UNSUPPORTED;  // B*H*N above 2^21
+    const safe_status st = noalloc_scratch(&ws);
+    if (st != SAFE_OK) return st;
+    ws_bytes = sizeof(g_pcsp_noalloc_scratch);
+  }
+  // Every element of the [B, H, N] partial block is written by the scoring
+  // kernel before the head sum reads it, so nothing needs clearing.
+  return safe_pcsp_topk(Q, Ky, valid_len, w, B, N, M, H, d, scale, scores, accumulate, k, S, C, ws, ws_bytes,
+                        stream);
 }
 
 safe_status safe_ctx_cache_scatter(const void* Ksrc, const void* Vsrc, int src_compact, const int32_t* S, int k,

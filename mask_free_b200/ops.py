@@ -39,6 +39,7 @@ _SIGS = {
     "safe_get_device_status": [ctypes.POINTER(ctypes.c_int), _vp],
     "safe_status_string": [_i],
     "safe_selftest_wait_timeout": [ctypes.c_uint64, _vp],
+    "safe_pcsp_topk_noalloc": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
 }
 _RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_status_string": ctypes.c_char_p}
 
