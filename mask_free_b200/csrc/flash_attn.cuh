@@ -9,19 +9,36 @@
 // One CTA owns two 128-row query tiles of one (b, h) and streams the key /
 // value tiles of that head through a shared-memory ring:
 //   warp 0       TMA producer (Q tiles once, then K_j / V_j per stage)
-//   warp 1       MMA issuer (one thread): S_t = Q_t K_j^T into TMEM, then
-//                O_t += P_t V_j with P_t read from TMEM (TS form)
-//   warps 2..5   softmax for tile 0, warps 6..9 softmax for tile 1: each
-//                thread owns one query row (one TMEM lane), reads S_t, keeps
-//                the running max / sum in registers, writes P_t (bf16) back
-//                into TMEM over S_t, rescales O_t lazily, and finally writes
-//                O = O_t / l (bf16) and the log-sum-exp.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D).
+//   warps 1, 2   MMA issuers (one thread each; tile 0 / tile 1): S_t = Q_t K_j^T
+//                into TMEM (SS form), O_t += P_t V_j with P read from TMEM
+//                (TS form). With D = 128 warp 1 issues for both tiles.
+//   warp 3       idle (it completes warpgroup 0)
+//   warps 4..7   softmax of tile 0, warps 8..11 softmax of tile 1: one
+//                thread per query row (one TMEM lane); running max / sum in
+//                registers; O rescaled lazily; final O = O_t / l (bf16) and
+//                the log-sum-exp.
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
+// O1 [256+D,256+2D) and, for D <= 96, one 64-column P buffer after O1 shared
+// by the two tiles. With the separate P buffer the softmax releases S_t as
+// soon as it has loaded it, so S_t for the next key tile is computed while
+// the softmax is still exponentiating; the P buffer alternates strictly
+// P0_j, P1_j, P0_{j+1}, ... (each write waits for the other tile's previous
+// P V product). For D = 128 there is no room for it: P overwrites S_t and the
+// next S_t is issued after P_t V.
+//
 // Online softmax in base 2: p = 2^(s*scale*log2(e) - m); O is only rescaled
 // when the running max grows by more than 8 (p stays below 2^8 otherwise).
 #pragma once
 
 #include "sm100.cuh"
+
+// Pairs of probabilities whose 2^x is evaluated by the FMA-pipe polynomial
+// instead of the MUFU unit: bit i of the mask selects pair i of every
+// 16-pair (32-column) chunk of a row.
+#ifndef SAFE_EXP_EMU_MASK
+#define SAFE_EXP_EMU_MASK 0x0000u
+#endif
 
 namespace safe {
 
@@ -31,12 +48,24 @@ struct TileCfg {
   static constexpr int kChunks = (D + 63) / 64;
   static constexpr int kTileBytes = 128 * D * 2;  // 128 rows of D bf16
   static constexpr int kStages = D <= 64 ? 4 : (D <= 96 ? 3 : 2);
-  // chunk c holds columns [64c, 64c + width(c)); 64-wide chunks use the 128B
-  // swizzle (128-byte rows), the 32-wide tail of D = 96 the 64B swizzle.
+  // Q and K tiles (K-major operands): chunk c holds columns [64c, 64c +
+  // width(c)); 64-wide chunks use the 128B swizzle (128-byte rows), the
+  // 32-wide tail of D = 96 the 64B swizzle.
   __host__ __device__ static constexpr int width(int c) { return (D - 64 * c) >= 64 ? 64 : (D - 64 * c); }
   __host__ __device__ static constexpr int row_bytes(int c) { return width(c) * 2; }
   __host__ __device__ static constexpr uint32_t chunk_off(int c) { return static_cast<uint32_t>(c) * 128u * 128u; }
   __host__ __device__ static constexpr uint32_t swizzle(int c) { return width(c) == 64 ? kSwizzle128B : kSwizzle64B; }
+  // V tiles (B operand of P V, MN-major) use equal-width chunks so that one
+  // MMA with N = D covers the whole head dim: 32-wide with the 64B swizzle
+  // for D = 96, 64-wide with the 128B swizzle otherwise; the descriptor's
+  // leading byte offset steps from one chunk to the next.
+  static constexpr int kVW = (D == 96) ? 32 : 64;
+  static constexpr int kVChunks = D / kVW;
+  static constexpr uint32_t kVChunkBytes = 128u * kVW * 2u;
+  static constexpr uint32_t kVSwizzle = kVW == 32 ? kSwizzle64B : kSwizzle128B;
+  // TMEM columns
+  static constexpr bool kSepP = 256 + 2 * D + 64 <= 512;
+  static constexpr uint32_t kColO = 256, kColP = 256 + 2 * D;
 };
 
 // K-major operand (rows of a 128-row tile, contiguous along the head dim):
@@ -50,19 +79,19 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 }
 
 // MN-major B operand (V tile: rows = keys, contiguous along the head dim):
-// descriptor of chunk c for the 16-key step kk.
+// descriptor of the 16-key step kk covering all D columns.
 template <int D>
-__device__ __forceinline__ uint64_t vmajor_desc(uint32_t tile, int c, int kk) {
+__device__ __forceinline__ uint64_t vmajor_desc(uint32_t tile, int kk) {
   using C = TileCfg<D>;
-  return make_sdesc(tile + C::chunk_off(c) + static_cast<uint32_t>(kk * 16 * C::row_bytes(c)), C::chunk_off(1),
-                    8 * C::row_bytes(c), C::swizzle(c));
+  return make_sdesc(tile + static_cast<uint32_t>(kk * 16 * C::kVW * 2), C::kVChunkBytes, 8 * C::kVW * 2,
+                    C::kVSwizzle);
 }
 
 struct FlashParams {
   CUtensorMap q_map[2];   // 4-D [B, rows, H, D] map per chunk (dense / compact Q)
   CUtensorMap qg_map[2];  // 2-D [B*N, H*D] gather map per chunk (rows of S)
   CUtensorMap k_map[2];   // 4-D [B, N, H, D]
-  CUtensorMap v_map[2];
+  CUtensorMap v_map;      // 4-D [B, N, H, D] V map, box kVW wide (chunk chosen by x)
   const int32_t* S;       // [B, n_q] query rows when gathering, else null
   __nv_bfloat16* O;       // [B, n_q, H, D]
   float* lse;             // [B, H, n_q] or null
@@ -71,7 +100,11 @@ struct FlashParams {
   int gather;
 };
 
-constexpr int kFlashThreads = 320;
+constexpr int kFlashThreads = 384;
+// Register split after setmaxnreg: warpgroup 0 (producer, MMA issuer) keeps
+// 104, the two softmax warpgroups get 200: 128*104 + 256*200 = 384*168, the
+// allocation the kernel is launched with (168 per thread).
+constexpr uint32_t kRegsControl = 104, kRegsSoftmax = 200;
 
 template <int D>
 __host__ __device__ constexpr int flash_smem_bytes() {
@@ -87,11 +120,18 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
+// Warp-uniform bounded wait (every lane polls; all agree on the outcome
+// before a warp-collective tcgen05 instruction follows).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __grid_constant__ FlashParams p) {
   using C = TileCfg<D>;
   constexpr int ST = C::kStages;
   constexpr int TB = C::kTileBytes;
+  constexpr bool kSepP = C::kSepP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm;
@@ -102,11 +142,13 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   uint64_t* k_full = q_full + 1;
   uint64_t* v_full = k_full + ST;
   uint64_t* kv_empty = v_full + ST;
-  uint64_t* s_full = kv_empty + ST;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
-  uint64_t* drain = o_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* s_full = kv_empty + ST;  // [2] S_t computed
+  uint64_t* s_free = s_full + 2;     // [2] S_t loaded by the softmax (separate-P mode)
+  uint64_t* p_full = s_free + 2;     // [2] P_t written
+  uint64_t* pv_done = p_full + 2;    // [2] P_t V complete
+  uint64_t* o_full = pv_done + 2;    // [2] last P_t V complete
+  uint64_t* drain = o_full + 2;      // [2] per MMA issuer, abort path only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -120,14 +162,17 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
     for (int s = 0; s < ST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], kSepP ? 2 : 1);  // one commit per MMA issuer
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
       mbar_init(&p_full[t], 128);
+      mbar_init(&pv_done[t], 1);
       mbar_init(&o_full[t], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
@@ -136,146 +181,194 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_prefetch_desc(&p.k_map[c]);
-        tma_prefetch_desc(&p.v_map[c]);
-      }
-      mbar_arrive_expect_tx(q_full, 2 * TB);
-    }
-    __syncwarp();
-    if (!p.gather) {
+  if (warp < 4) {
+    regs_dealloc<kRegsControl>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
       if (lane == 0) {
-        for (int t = 0; t < 2; ++t)
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_4d(sQ + t * TB + C::chunk_off(c), &p.q_map[c], q_full, 64 * c, h, q_base + t * 128, b);
+        for (int c = 0; c < C::kChunks; ++c) tma_prefetch_desc(&p.k_map[c]);
+        tma_prefetch_desc(&p.v_map);
+        mbar_arrive_expect_tx(q_full, 2 * TB);
       }
-    } else {
-      // lane l gathers rows 4l..4l+3 of each tile (indices clamped to the
-      // last valid row for the ragged tail; out-of-range indices flagged)
-      for (int t = 0; t < 2; ++t) {
-        int y[4];
-        for (int u = 0; u < 4; ++u) {
-          int r = q_base + t * 128 + 4 * lane + u;
-          r = r < p.n_q ? r : p.n_q - 1;
-          int idx = __ldg(p.S + static_cast<size_t>(b) * p.n_q + r);
-          if (idx < 0 || idx >= p.N) {
-            raise_status(1 << 5);
-            idx = 0;
+      __syncwarp();
+      if (!p.gather) {
+        if (lane == 0) {
+          for (int t = 0; t < 2; ++t)
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(sQ + t * TB + C::chunk_off(c), &p.q_map[c], q_full, 64 * c, h, q_base + t * 128, b);
+        }
+      } else {
+        // lane l gathers rows 4l..4l+3 of each tile (indices clamped to the
+        // last valid row for the ragged tail; out-of-range indices flagged)
+        for (int t = 0; t < 2; ++t) {
+          int y[4];
+          for (int u = 0; u < 4; ++u) {
+            int r = q_base + t * 128 + 4 * lane + u;
+            r = r < p.n_q ? r : p.n_q - 1;
+            int idx = __ldg(p.S + static_cast<size_t>(b) * p.n_q + r);
+            if (idx < 0 || idx >= p.N) {
+              raise_status(1 << 5);
+              idx = 0;
+            }
+            y[u] = b * p.N + idx;
           }
-          y[u] = b * p.N + idx;
-        }
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_gather4(sQ + t * TB + C::chunk_off(c) + 4 * lane * C::row_bytes(c), &p.qg_map[c], q_full,
-                      h * D + 64 * c, y[0], y[1], y[2], y[3]);
-      }
-    }
-    if (lane == 0) {
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % ST;
-        if (j >= ST && !mbar_wait(&kv_empty[s], ((j / ST) - 1) & 1, &abort_flag)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&k_full[s], TB);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sK + s * TB + C::chunk_off(c), &p.k_map[c], &k_full[s], 64 * c, h, j * 128, b);
-        mbar_arrive_expect_tx(&v_full[s], TB);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sV + s * TB + C::chunk_off(c), &p.v_map[c], &v_full[s], 64 * c, h, j * 128, b);
-        issued = j + 1;
-      }
-      if (!ok || abort_flag) {
-        // let every copy this CTA started land before the CTA exits
-        mbar_wait_drain(q_full, 0);
-        for (int j = issued - ST < 0 ? 0 : issued - ST; j < issued; ++j) {
-          mbar_wait_drain(&k_full[j % ST], (j / ST) & 1);
-          mbar_wait_drain(&v_full[j % ST], (j / ST) & 1);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_gather4(sQ + t * TB + C::chunk_off(c) + 4 * lane * C::row_bytes(c), &p.qg_map[c], q_full,
+                        h * D + 64 * c, y[0], y[1], y[2], y[3]);
         }
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = make_idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idPV0 = make_idesc_bf16(128, C::width(0), 0, 1);
-      constexpr uint32_t idPV1 = make_idesc_bf16(128, C::kChunks > 1 ? C::width(1) : 64, 0, 1);
-      const uint32_t tS[2] = {tbase, tbase + 128};
-      const uint32_t tO[2] = {tbase + 256, tbase + 256 + D};
-      const uint32_t aQ[2] = {smem_u32(sQ), smem_u32(sQ + TB)};
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-      auto issue_S = [&](int t, int s) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tS[t], kmajor_desc<D>(aQ[t], kk), kmajor_desc<D>(aK + s * TB, kk), idS, kk > 0 ? 1u : 0u);
-      };
-      auto issue_PV = [&](int t, int s, int j) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          umma_ts(tO[t], tS[t] + kk * 8, vmajor_desc<D>(aV + s * TB, 0, kk), idPV0, acc);
-          if (C::kChunks > 1)
-            umma_ts(tO[t] + 64, tS[t] + kk * 8, vmajor_desc<D>(aV + s * TB, 1, kk), idPV1, acc);
-        }
-      };
-      bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&k_full[0], 0, &abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_S(0, 0);
-        umma_commit(&s_full[0]);
-        issue_S(1, 0);
-        umma_commit(&s_full[1]);
-        for (int j = 0; j < n_kv && ok; ++j) {
+      if (lane == 0) {
+        int issued = 0;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
           const int s = j % ST;
-          ok = mbar_wait(&v_full[s], (j / ST) & 1, &abort_flag);
-          for (int t = 0; t < 2 && ok; ++t) {
-            ok = mbar_wait(&p_full[t], j & 1, &abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_PV(t, s, j);
-            if (j + 1 < n_kv) {
-              const int s1 = (j + 1) % ST;
-              if (t == 0) {
-                ok = mbar_wait(&k_full[s1], ((j + 1) / ST) & 1, &abort_flag);
+          if (j >= ST && !mbar_wait(&kv_empty[s], ((j / ST) - 1) & 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[s], TB);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sK + s * TB + C::chunk_off(c), &p.k_map[c], &k_full[s], 64 * c, h, j * 128, b);
+          mbar_arrive_expect_tx(&v_full[s], TB);
+          for (int c = 0; c < C::kVChunks; ++c)
+            tma_load_4d(sV + s * TB + c * C::kVChunkBytes, &p.v_map, &v_full[s], C::kVW * c, h, j * 128, b);
+          issued = j + 1;
+        }
+        if (!ok || abort_flag) {
+          // let every copy this CTA started land before the CTA exits
+          mbar_wait_drain(q_full, 0);
+          for (int j = issued - ST < 0 ? 0 : issued - ST; j < issued; ++j) {
+            mbar_wait_drain(&k_full[j % ST], (j / ST) & 1);
+            mbar_wait_drain(&v_full[j % ST], (j / ST) & 1);
+          }
+        }
+      }
+    } else if (warp == 1 || (kSepP && warp == 2)) {
+      // ---------------------------------------------------------- MMA issuers
+      // separate-P mode: warp 1 issues tile 0's MMAs and warp 2 tile 1's
+      // (tcgen05.commit tracks the issuing thread's MMAs, so each issuer
+      // signals its own tile); aliased mode: warp 1 issues both tiles.
+      if (lane == 0) {
+        const int mt = warp - 1;  // tile of this issuer (separate-P mode)
+        constexpr uint32_t idS = make_idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idPV = make_idesc_bf16(128, D, 0, 1);
+        constexpr int KS = D / 16;
+        // TMEM column of S_t, O_t and P_t (t = 0, 1)
+        auto tS = [&](int t) -> uint32_t { return tbase + 128u * t; };
+        auto tO = [&](int t) -> uint32_t { return tbase + C::kColO + static_cast<uint32_t>(D) * t; };
+        auto tP = [&](int t) -> uint32_t { return kSepP ? tbase + C::kColP : tbase + 128u * t; };
+        // Descriptors of stage 0 / k-step 0; a k-step or a stage only moves
+        // the start address (low 14 bits, in 16-byte units), so each MMA
+        // adds a constant to the low word.
+        const uint64_t dQ0 = kmajor_desc<D>(smem_u32(sQ), 0), dQ1 = kmajor_desc<D>(smem_u32(sQ + TB), 0);
+        const uint64_t dK = kmajor_desc<D>(smem_u32(sK), 0);
+        const uint64_t dV = vmajor_desc<D>(smem_u32(sV), 0);
+        auto koff = [](int kk) -> uint32_t { return (C::chunk_off(kk >> 2) + (kk & 3) * 32) >> 4; };
+        // the two K-major chunks of D = 96 differ in swizzle: take the high
+        // word (layout, strides) per chunk, the start address from the base
+        auto kdesc = [&](uint64_t base, int kk, uint32_t so) -> uint64_t {
+          const uint64_t hi = kmajor_desc<D>(0, kk) & 0xFFFFFFFF00000000ull;
+          return hi | static_cast<uint32_t>(static_cast<uint32_t>(base) + koff(kk) + so);
+        };
+        auto issue_S = [&](int t, int s) {
+          const uint32_t so = static_cast<uint32_t>((s * TB) >> 4);
+          const uint64_t dq = t == 0 ? dQ0 : dQ1;
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) umma_ss(tS(t), kdesc(dq, kk, 0), kdesc(dK, kk, so), idS, kk > 0 ? 1u : 0u);
+        };
+        // O_t (+)= P_t V: 8 steps of 16 keys, one N = D instruction each
+        auto issue_PV = [&](int t, int s, int j) {
+          const uint32_t so = static_cast<uint32_t>((s * TB) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t v = static_cast<uint32_t>(dV) + so + ((kk * 16 * C::kVW * 2) >> 4);
+            umma_ts(tO(t), tP(t) + kk * 8, (dV & 0xFFFFFFFF00000000ull) | v, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        };
+        bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&k_full[0], 0, &abort_flag);
+        if (ok) {
+          tc_fence_after();
+          if constexpr (kSepP) {
+            // per tile: the next S as soon as the softmax has loaded the
+            // current one, then P V once P is written
+            issue_S(mt, 0);
+            umma_commit(&s_full[mt]);
+            for (int j = 0; j < n_kv && ok; ++j) {
+              const int s = j % ST;
+              if (j + 1 < n_kv) {
+                const int s1 = (j + 1) % ST;
+                ok = mbar_wait(&k_full[s1], ((j + 1) / ST) & 1, &abort_flag) &&
+                     mbar_wait(&s_free[mt], j & 1, &abort_flag);
                 if (!ok) break;
                 tc_fence_after();
+                issue_S(mt, s1);
+                umma_commit(&s_full[mt]);
               }
-              issue_S(t, s1);
-              umma_commit(&s_full[t]);
-            } else {
-              umma_commit(&o_full[t]);
+              ok = mbar_wait(&v_full[s], (j / ST) & 1, &abort_flag) && mbar_wait(&p_full[mt], j & 1, &abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              issue_PV(mt, s, j);
+              umma_commit(&pv_done[mt]);
+              umma_commit(&kv_empty[s]);  // this tile no longer reads K_j, V_j
+              if (j + 1 == n_kv) umma_commit(&o_full[mt]);
             }
+          } else {
+          issue_S(0, 0);
+          umma_commit(&s_full[0]);
+          issue_S(1, 0);
+          umma_commit(&s_full[1]);
+          for (int j = 0; j < n_kv && ok; ++j) {
+            const int s = j % ST;
+            {
+              // P overwrites S_t: the next S_t follows P_t V
+              ok = mbar_wait(&v_full[s], (j / ST) & 1, &abort_flag);
+              for (int t = 0; t < 2 && ok; ++t) {
+                ok = mbar_wait(&p_full[t], j & 1, &abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                issue_PV(t, s, j);
+                if (j + 1 < n_kv) {
+                  const int s1 = (j + 1) % ST;
+                  if (t == 0) {
+                    ok = mbar_wait(&k_full[s1], ((j + 1) / ST) & 1, &abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                  }
+                  issue_S(t, s1);
+                  umma_commit(&s_full[t]);
+                } else {
+                  umma_commit(&o_full[t]);
+                }
+              }
+            }
+            if (ok) umma_commit(&kv_empty[s]);
           }
-          if (ok) umma_commit(&kv_empty[s]);
+          }
         }
-      }
-      if (!ok) {
-        // wait for every MMA this thread issued before TMEM is released
-        umma_commit(drain);
-        mbar_wait_drain(drain, 0);
+        if (!ok) {
+          // wait for every MMA this thread issued before TMEM is released
+          umma_commit(&drain[warp - 1]);
+          mbar_wait_drain(&drain[warp - 1], 0);
+        }
       }
     }
   } else {
+    regs_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;
+    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tbase + lane_addr + t * 128;
-    const uint32_t tO = tbase + lane_addr + 256 + t * D;
+    const uint32_t tO = tbase + lane_addr + C::kColO + t * D;
+    const uint32_t tP = kSepP ? tbase + lane_addr + C::kColP : tS;
     const int q_row = q_base + t * 128 + row;
     const float sl2 = p.scale_log2;
     const int tail = p.N - (n_kv - 1) * 128;  // valid keys in the last tile
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      // every lane waits; the outcome is made warp-uniform before the
-      // warp-collective tcgen05.ld below
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, &abort_flag))) {
+      if (!warp_wait(&s_full[t], j & 1, &abort_flag)) {
         ok = false;
         break;
       }
@@ -289,21 +382,30 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       tmem_ld_wait32(sr + 32);
       tmem_ld_wait32(sr + 64);
       tmem_ld_wait32(sr + 96);
+      if constexpr (kSepP) {
+        // S_t is in registers: the MMA issuer may overwrite it
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);
+      }
       if (j == n_kv - 1 && tail < 128) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= tail) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+      float mx0 = fmax3(__uint_as_float(sr[0]), __uint_as_float(sr[1]), __uint_as_float(sr[2]));
+      float mx1 = fmax3(__uint_as_float(sr[3]), __uint_as_float(sr[4]), __uint_as_float(sr[5]));
+      float mx2 = fmax3(__uint_as_float(sr[6]), __uint_as_float(sr[7]), __uint_as_float(sr[8]));
+      float mx3 = fmax3(__uint_as_float(sr[9]), __uint_as_float(sr[10]), __uint_as_float(sr[11]));
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+      for (int c = 12; c < 124; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
       }
-      const float m_cand = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      mx0 = fmax3(mx0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
+      mx1 = fmax3(mx1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+      const float m_cand = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
       float alpha = 1.f;
       bool need = false;
       if (j == 0) {
@@ -315,40 +417,62 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
           m_use = m_cand;
         }
       }
-      const float neg = -m_use;
-      float sum0 = 0.f, sum1 = 0.f;
+      // probabilities (bf16 pairs) and the row sum
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc0 = 0, acc1 = 0;  // packed row sums (bit pattern 0 = +0.0f)
+      uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = ex2_approx(fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, neg));
-          const float bb = ex2_approx(fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, neg));
-          sum0 += a;
-          sum1 += bb;
-          pk[i] = pack_bf16x2(a, bb);
-        }
-        tmem_st16(tS + 16 * c, pk);
+      for (int i = 0; i < 64; ++i) {
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm2);
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        uint64_t e2;
+        if ((SAFE_EXP_EMU_MASK >> (i & 15)) & 1u)
+          e2 = exp2_poly_f2(x0, x1);
+        else
+          e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        if (i & 1) acc1 = f2_add(acc1, e2); else acc0 = f2_add(acc0, e2);
+        float a, bb;
+        f2_unpack(e2, a, bb);
+        pk[i] = pack_bf16x2(a, bb);
       }
-      // O_t is idle here (PV_t of the previous step completed before S_t of
-      // this step was committed), so the rescale can follow the P store.
+      if constexpr (kSepP) {
+        // P buffer turn: P0_j follows P1_{j-1} V, P1_j follows P0_j V. That
+        // wait also orders this tile's previous P V before the O rescale.
+        bool turn = true;
+        if (t == 0 && j > 0) turn = warp_wait(&pv_done[1], (j - 1) & 1, &abort_flag);
+        if (t == 1) turn = warp_wait(&pv_done[0], j & 1, &abort_flag);
+        if (!turn) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      // (aliased mode: O_t is idle because P_t V of the previous step
+      // completed before S_t of this step was committed)
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_ld_wait32(o);
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16 * c, o);
+          tmem_ld_wait16(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * c, o);
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16(tO + 16 * c, o);
         }
       }
-      l = l * alpha + (sum0 + sum1);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
+      float s0, s1, s2, s3;
+      f2_unpack(acc0, s0, s1);
+      f2_unpack(acc1, s2, s3);
+      l = l * alpha + ((s0 + s1) + (s2 + s3));
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, &abort_flag))) {
+    if (ok && warp_wait(&o_full[t], 0, &abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool valid = q_row < p.n_q;

@@ -71,6 +71,23 @@ bool encode_rows_map(CUtensorMap* map, const void* base, int B, int rows, int H,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Same 4-D view with the equal-width V chunks of the flash kernel (32 wide
+// with the 64B swizzle for d = 96, else 64 wide with the 128B swizzle).
+bool encode_v_map(CUtensorMap* map, const void* base, int B, int rows, int H, int d) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const int w = d == 96 ? 32 : 64;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                           static_cast<cuuint64_t>(rows) * H * d * 2};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(w), 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, w == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [B*N, H*d] 2-D view for tile::gather4 (box one row high).
 bool encode_gather_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int c) {
   auto fn = encode_fn();
@@ -272,10 +289,10 @@ safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O,
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
   for (int c = 0; c < nchunks(d); ++c) {
-    if (!encode_rows_map(&p.q_map[c], Q, B, N, H, d, c) || !encode_rows_map(&p.k_map[c], K, B, N, H, d, c) ||
-        !encode_rows_map(&p.v_map[c], V, B, N, H, d, c))
+    if (!encode_rows_map(&p.q_map[c], Q, B, N, H, d, c) || !encode_rows_map(&p.k_map[c], K, B, N, H, d, c))
       return SAFE_ERR_CUDA;
   }
+  if (!encode_v_map(&p.v_map, V, B, N, H, d)) return SAFE_ERR_CUDA;
   p.S = nullptr;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.lse = lse;
@@ -295,8 +312,9 @@ safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k
   if (!q_compact && S == nullptr) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
+  if (!encode_v_map(&p.v_map, Vc, B, N, H, d)) return SAFE_ERR_CUDA;
   for (int c = 0; c < nchunks(d); ++c) {
-    bool ok = encode_rows_map(&p.k_map[c], Kc, B, N, H, d, c) && encode_rows_map(&p.v_map[c], Vc, B, N, H, d, c);
+    bool ok = encode_rows_map(&p.k_map[c], Kc, B, N, H, d, c);
     ok = ok && (q_compact ? encode_rows_map(&p.q_map[c], Q, B, k, H, d, c)
                           : encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c));
     if (!ok) return SAFE_ERR_CUDA;

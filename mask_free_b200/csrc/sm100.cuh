@@ -60,20 +60,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase `parity` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on phase `parity`. `abort` is a CTA-shared flag: when another
 // role of the CTA has given up, this wait gives up too. Returns true when the
-// phase completed.
+// phase completed. The limit is measured on %globaltimer, read only every
+// 256 polls so that the polling loop stays short.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  for (uint32_t polls = 1;; ++polls) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      *abort = 1;
-      raise_status(1 << 4);  // SAFE_ERR_TIMEOUT
-      return false;
+    if ((polls & 255u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        raise_status(1 << 4);  // SAFE_ERR_TIMEOUT
+        return false;
+      }
     }
   }
 }
@@ -246,5 +262,65 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __device__ __forceinline__ uint32_t elect_one_lane() { return (threadIdx.x & 31) == 0; }
+
+// ---------------------------------------------------------------- register reconfiguration
+// Warpgroup-wide: every warp of the warpgroup executes it.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------- packed fp32 (sm_100 f32x2)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair on the FMA pipe (Cody-Waite split x = n + f with n the
+// nearest integer, then a degree-3 minimax polynomial for 2^f on
+// [-1/2, 1/2] fitted by iteratively reweighted least squares; max relative
+// error 8.4e-5, far below the bf16 rounding of the probabilities). x is
+// clamped to >= -126 so the exponent add cannot wrap; results below 2^-126
+// are negligible next to the row sum.
+__device__ __forceinline__ uint64_t exp2_poly_f2(float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t r = f2_add(t, f2_pack(-kShift, -kShift));                       // round(x)
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);                          // x - round(x)
+  uint64_t p = f2_fma(f2_pack(0.055213045f, 0.055213045f), f, f2_pack(0.24271424f, 0.24271424f));
+  p = f2_fma(p, f, f2_pack(0.69326216f, 0.69326216f));
+  p = f2_fma(p, f, f2_pack(0.99991959f, 0.99991959f));
+  // scale by 2^n: add n to the exponent field (t's low mantissa bits hold n)
+  const uint32_t t0 = static_cast<uint32_t>(t), t1 = static_cast<uint32_t>(t >> 32);
+  const uint32_t p0 = static_cast<uint32_t>(p), p1 = static_cast<uint32_t>(p >> 32);
+  const uint32_t e0 = p0 + (t0 << 23), e1 = p1 + (t1 << 23);
+  return (static_cast<uint64_t>(e1) << 32) | e0;
+}
 
 }  // namespace safe
