@@ -37,7 +37,9 @@ from mask_free_b200 import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s + ms/call (dense, SRSU) at N=4096/25600; % bf16 tensor peak"
 WORKLOAD = "2560^2-equivalent SRSU step: B=2, H=24, d=96, N=25600, M=128 (len U[8,128]), k=6400 (0.25N)"
-LAUNCHES_PER_STEP = 11  # classify 3, self 1, cross 1, pcsp 3 (scores, head sum, top-k), scatter 1, srsu 1, cross(S) 1
+# classify 3, self 1 (+1 workspace-counter reset when the key split is used), cross 1, pcsp 3 (scores,
+# head sum, top-k), scatter 1, srsu 1 (+1), cross(S) 1
+LAUNCHES_PER_STEP = 11
 
 
 def peaks():
@@ -163,6 +165,8 @@ class Step:
         self.C = torch.empty((B, N - k), dtype=torch.int32, device=dev)
         self.ws = torch.empty(ops.pcsp_workspace_bytes(B, N, H), dtype=torch.uint8, device=dev)
         self.cls = torch.empty(3, dtype=torch.int64, device=dev)
+        self.ws_self = torch.empty(max(256, ops.attn_workspace_bytes(B, N, N, H, d)), dtype=torch.uint8, device=dev)
+        self.ws_srsu = torch.empty(max(256, ops.attn_workspace_bytes(B, k, N, H, d)), dtype=torch.uint8, device=dev)
         self.Kc, self.Vc = inp["Kc"].clone(), inp["Vc"].clone()
         self.events = []
 
@@ -174,7 +178,7 @@ class Step:
         o.mask_classify(i["mask"], sync=False, result=self.cls)
         if timed:
             ev[0].record()
-        o.attn_self(i["Q"], i["K"], i["V"], out=self.O)
+        o.attn_self(i["Q"], i["K"], i["V"], out=self.O, ws=self.ws_self)
         if timed:
             ev[1].record()
         o.attn_cross(i["Q"], i["Ky"], i["Vy"], i["valid_len"], out=self.Ox)
@@ -183,7 +187,7 @@ class Step:
         o.ctx_cache_scatter(i["K"], i["V"], self.S, self.Kc, self.Vc, src_compact=False)
         if timed:
             ev[2].record()
-        o.srsu_attn(i["Q"], self.S, self.Kc, self.Vc, out=self.Os)
+        o.srsu_attn(i["Q"], self.S, self.Kc, self.Vc, out=self.Os, ws=self.ws_srsu)
         if timed:
             ev[3].record()
         o.attn_cross(i["Q"], i["Ky"], i["Vy"], i["valid_len"], q_idx=self.S, out=self.Osx)
@@ -222,8 +226,10 @@ def kernel_table(dev, pk):
         O = torch.empty_like(inp["Q"])
         Os = torch.empty((s.B, k, s.H, s.d), dtype=torch.bfloat16, device=dev)
         dense_f, srsu_f, cross_f, _ = flops(s, lsum, k)
-        t_d = time_kernel(lambda: ops.attn_self(inp["Q"], inp["K"], inp["V"], out=O))
-        t_s = time_kernel(lambda: ops.srsu_attn(inp["Q"], S, inp["Kc"], inp["Vc"], out=Os))
+        ws_d = torch.empty(max(256, ops.attn_workspace_bytes(s.B, s.N, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
+        ws_s = torch.empty(max(256, ops.attn_workspace_bytes(s.B, k, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
+        t_d = time_kernel(lambda: ops.attn_self(inp["Q"], inp["K"], inp["V"], out=O, ws=ws_d))
+        t_s = time_kernel(lambda: ops.srsu_attn(inp["Q"], S, inp["Kc"], inp["Vc"], out=Os, ws=ws_s))
         Ox = torch.empty_like(O)
         t_x = time_kernel(lambda: ops.attn_cross(inp["Q"], inp["Ky"], inp["Vy"], inp["valid_len"], out=Ox))
         tag = f"N{s.N}"
@@ -261,8 +267,10 @@ def kernel_table(dev, pk):
                 kk = max(1, math.ceil(rho * s.N))
                 Sr = torch.sort(torch.randperm(s.N, device=dev)[:kk])[0].to(torch.int32).expand(s.B, kk).contiguous()
                 Osr = torch.empty((s.B, kk, s.H, s.d), dtype=torch.bfloat16, device=dev)
-                sweep[str(rho)] = time_kernel(lambda: ops.srsu_attn(inp["Q"], Sr, inp["Kc"], inp["Vc"], out=Osr),
-                                              reps=10)
+                wsr = torch.empty(max(256, ops.attn_workspace_bytes(s.B, kk, s.N, s.H, s.d)), dtype=torch.uint8,
+                                  device=dev)
+                sweep[str(rho)] = time_kernel(lambda: ops.srsu_attn(inp["Q"], Sr, inp["Kc"], inp["Vc"], out=Osr,
+                                                                    ws=wsr), reps=10)
             out["srsu_rho_sweep_ms"] = sweep
             out["srsu_t_rho_over_t_1"] = {r: v / sweep["1.0"] for r, v in sweep.items()}
         del inp

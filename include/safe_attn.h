@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { SAFE_BOOL = 0, SAFE_U8 = 1, SAFE_F32 = 2, SAFE_F16 = 3, SAFE_BF16 = 4 } safe_dtype;
 
-/* ABI version of this header (bumped on any signature change). */
+/* ABI version of this header (bumped on any signature change): 2. */
 int safe_abi_version(void);
 const char* safe_status_string(int status);
 
@@ -94,10 +94,18 @@ safe_status safe_mask_classify_sync(const void* mask, int dtype, const int64_t s
  *  Q, K, V  device bf16 [B, N, H, d];  O device bf16 [B, N, H, d] (written).
  *  lse      device fp32 [B, H, N] natural-log log-sum-exp of the scaled
  *           logits, or NULL.
+ *  ws       device workspace of safe_attn_workspace_bytes(B, N, N, H, d)
+ *           bytes (256-byte aligned), or NULL. With it, the units of the
+ *           last, partial wave of CTAs are split into key ranges whose
+ *           partial results a second small kernel merges (balances the
+ *           wave); without it every CTA takes all keys. Either way the
+ *           result is the same up to fp32 rounding order. Contents need no
+ *           initialisation; the size is 0 when no split pays off.
  * fp32 accumulation and softmax; O is rounded to bf16 (nearest even).
  */
+size_t safe_attn_workspace_bytes(int B, int n_q, int N, int H, int d);
 safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O, float* lse, int B, int N, int H,
-                           int d, float scale, void* stream);
+                           int d, float scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Image->text cross-attention keeping the text padding mask, Eq. (4), and its
@@ -190,9 +198,11 @@ safe_status safe_topk_partition(const float* scores, int B, int N, int k, int32_
  *  S        device int32 [B, k], strictly ascending, values in [0, N).
  *  Kc, Vc   device bf16 [B, N, H, d].
  *  O_S      device bf16 [B, k, H, d] (written); lse device fp32 [B, H, k] or NULL.
+ *  ws       as safe_attn_self, sized safe_attn_workspace_bytes(B, k, N, H, d).
  */
 safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
-                           void* O_S, float* lse, int B, int N, int H, int d, float scale, void* stream);
+                           void* O_S, float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
+                           void* stream);
 
 /*
  * Context-cache update, Eq. (14), (16), (19): write the current sensitive

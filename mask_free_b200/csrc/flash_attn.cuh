@@ -98,6 +98,14 @@ struct FlashParams {
   int B, N, H, n_q;
   float scale_log2;       // logit scale * log2(e)
   int gather;
+  // Work units are (b, h, 256-row block), ordered with the row block
+  // fastest. The first `full_units` CTAs take one whole unit each; the
+  // remaining units are split along the key range into `split` parts, one
+  // CTA each, whose partial results flash_merge_kernel combines (balances
+  // the last, partial wave of CTAs).
+  int n_mblk, full_units, split;
+  float* ws_o;            // [tail units][split][256][D] unnormalised partial O
+  float2* ws_ml;          // [tail units][split][256] (running max in log2 units, row sum)
 };
 
 constexpr int kFlashThreads = 384;
@@ -110,6 +118,49 @@ template <int D>
 __host__ __device__ constexpr int flash_smem_bytes() {
   using C = TileCfg<D>;
   return 1024 /*align slack*/ + (2 + 2 * C::kStages) * C::kTileBytes + 256 /*barriers + tmem slot*/;
+}
+
+// Combines the key-range parts of the split units: one warp per query row,
+// lane l owns columns [4l, 4l + 4):
+//   M = max_i m_i,  L = sum_i 2^(m_i - M) l_i,  O = sum_i 2^(m_i - M) O_i / L
+template <int D>
+__global__ void __launch_bounds__(256) flash_merge_kernel(const __grid_constant__ FlashParams p, int tail_units) {
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (wid >= tail_units * 256) return;
+  const int tu = wid / 256, r = wid % 256;
+  const int unit = p.full_units + tu;
+  const int h = (unit / p.n_mblk) % p.H, b = unit / (p.n_mblk * p.H);
+  const int qr = (unit % p.n_mblk) * 256 + r;
+  if (qr >= p.n_q) return;
+  const size_t slot0 = static_cast<size_t>(tu) * p.split * 256 + r;
+  float M = -INFINITY;
+  for (int i = 0; i < p.split; ++i) M = fmaxf(M, __ldcg(&p.ws_ml[slot0 + static_cast<size_t>(i) * 256]).x);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const bool active = lane < D / 4;
+#pragma unroll 4
+  for (int i = 0; i < p.split; ++i) {
+    const size_t slot = slot0 + static_cast<size_t>(i) * 256;
+    const float2 ml = __ldcg(&p.ws_ml[slot]);
+    const float w = ex2_approx(ml.x - M);
+    L = fmaf(w, ml.y, L);
+    if (active) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(p.ws_o + slot * D) + lane);
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z);
+      acc.w = fmaf(w, x.w, acc.w);
+    }
+  }
+  const float inv_l = 1.f / L;
+  if (active) {
+    __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.n_q + qr) * p.H + h) * D;
+    reinterpret_cast<uint2*>(orow)[lane] =
+        make_uint2(pack_bf16x2(acc.x * inv_l, acc.y * inv_l), pack_bf16x2(acc.z * inv_l, acc.w * inv_l));
+  }
+  if (lane == 0 && p.lse != nullptr)
+    p.lse[(static_cast<size_t>(b) * p.H + h) * p.n_q + qr] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
@@ -152,9 +203,20 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.z, h = blockIdx.y;
-  const int q_base = blockIdx.x * 256;
-  const int n_kv = (p.N + 127) / 128;
+  const int n_kv_all = (p.N + 127) / 128;
+  int unit = blockIdx.x, tail_u = 0, part = 0, kv0 = 0, kv1 = n_kv_all;
+  if (unit >= p.full_units) {
+    const int k = unit - p.full_units;
+    tail_u = k / p.split;
+    part = k % p.split;
+    unit = p.full_units + tail_u;
+    kv0 = part * n_kv_all / p.split;
+    kv1 = (part + 1) * n_kv_all / p.split;
+  }
+  const bool partial = p.split > 1 && blockIdx.x >= p.full_units;
+  const int h = (unit / p.n_mblk) % p.H, b = unit / (p.n_mblk * p.H);
+  const int q_base = (unit % p.n_mblk) * 256;
+  const int n_kv = kv1 - kv0;  // key tiles of this CTA: [kv0, kv1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -228,10 +290,10 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
           }
           mbar_arrive_expect_tx(&k_full[s], TB);
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_4d(sK + s * TB + C::chunk_off(c), &p.k_map[c], &k_full[s], 64 * c, h, j * 128, b);
+            tma_load_4d(sK + s * TB + C::chunk_off(c), &p.k_map[c], &k_full[s], 64 * c, h, (kv0 + j) * 128, b);
           mbar_arrive_expect_tx(&v_full[s], TB);
           for (int c = 0; c < C::kVChunks; ++c)
-            tma_load_4d(sV + s * TB + c * C::kVChunkBytes, &p.v_map, &v_full[s], C::kVW * c, h, j * 128, b);
+            tma_load_4d(sV + s * TB + c * C::kVChunkBytes, &p.v_map, &v_full[s], C::kVW * c, h, (kv0 + j) * 128, b);
           issued = j + 1;
         }
         if (!ok || abort_flag) {
@@ -364,7 +426,8 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
     const uint32_t tP = kSepP ? tbase + lane_addr + C::kColP : tS;
     const int q_row = q_base + t * 128 + row;
     const float sl2 = p.scale_log2;
-    const int tail = p.N - (n_kv - 1) * 128;  // valid keys in the last tile
+    // valid keys in this CTA's last tile (fewer than 128 only in the global last tile)
+    const int tail = kv1 == n_kv_all ? p.N - (n_kv_all - 1) * 128 : 128;
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
@@ -472,11 +535,12 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       f2_unpack(acc1, s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
     }
-    if (ok && warp_wait(&o_full[t], 0, &abort_flag)) {
-      tc_fence_after();
+    const bool have_o = ok && warp_wait(&o_full[t], 0, &abort_flag);
+    if (have_o) tc_fence_after();
+    const bool valid = q_row < p.n_q;
+    __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.n_q + (valid ? q_row : 0)) * p.H + h) * D;
+    if (have_o && !partial) {
       const float inv_l = 1.f / l;
-      const bool valid = q_row < p.n_q;
-      __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.n_q + (valid ? q_row : 0)) * p.H + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -494,6 +558,26 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       }
       if (valid && p.lse != nullptr)
         p.lse[(static_cast<size_t>(b) * p.H + h) * p.n_q + q_row] = (m_use + __log2f(l)) * 0.69314718055994531f;
+    }
+    if (partial) {
+      // one part of a split unit: store the unnormalised O row with its
+      // running max and sum (flash_merge_kernel combines the parts)
+      const size_t slot0 = static_cast<size_t>(tail_u) * p.split * 256 + t * 128 + row;
+      if (have_o) {
+        float* po = p.ws_o + (slot0 + static_cast<size_t>(part) * 256) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait32(o);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            reinterpret_cast<float4*>(po + 32 * c)[v] =
+                make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]), __uint_as_float(o[4 * v + 2]),
+                            __uint_as_float(o[4 * v + 3]));
+        }
+        p.ws_ml[slot0 + static_cast<size_t>(part) * 256] = make_float2(m_use, l);
+      }
     }
   }
 

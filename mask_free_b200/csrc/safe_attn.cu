@@ -21,7 +21,7 @@ using namespace safe;
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -104,8 +104,67 @@ bool encode_gather_map(CUtensorMap* map, const void* base, int B, int N, int H, 
 int nchunks(int d) { return (d + 63) / 64; }
 
 // ---------------------------------------------------------------- launches
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return sms;
+  static int cached[64] = {};
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = sms;
+  return sms;
+}
+
+// How the (b, h, 256-row block) work units of one flash launch are spread
+// over the SMs: `full` whole units first, then the remaining units split
+// into `split` key ranges each (see FlashParams).
+struct FlashPlan {
+  int units, full, split, tail;
+  size_t ws_o, ws_ml, ws_bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+FlashPlan plan_flash(int B, int H, int n_q, int N, int d, int sms) {
+  FlashPlan pl{};
+  const int n_mblk = (n_q + 255) / 256;
+  const int n_kv = (N + 127) / 128;
+  pl.units = n_mblk * H * B;
+  pl.full = pl.units;
+  pl.split = 1;
+  pl.tail = 0;
+  // Cost model in key-tile steps (calibrated on B200): a whole unit costs
+  // n_kv + 2, a part n_kv / s + 8 (set-up, pipeline fill and drain, partial
+  // store, and the spread of finish times across SMs), the merge launch
+  // about 3. Only the last waves are split; each part keeps at least 4 key
+  // tiles.
+  const double whole = n_kv + 2.0;
+  double best = static_cast<double>((pl.units + sms - 1) / sms) * whole;
+  const int max_split = n_kv / 4 < 16 ? n_kv / 4 : 16;
+  for (int fw = pl.units / sms; fw >= 0 && fw >= pl.units / sms - 1; --fw) {
+    const int f = fw * sms, r = pl.units - f;
+    if (r <= 0) continue;
+    for (int sp = 2; sp <= max_split; ++sp) {
+      const double rounds = static_cast<double>((static_cast<long long>(r) * sp + sms - 1) / sms);
+      const double cost = fw * whole + rounds * (static_cast<double>(n_kv) / sp + 8.0) + 3.0;
+      if (cost < 0.99 * best) {
+        best = cost;
+        pl.full = f;
+        pl.split = sp;
+        pl.tail = r;
+      }
+    }
+  }
+  if (pl.split > 1) {
+    const size_t slots = static_cast<size_t>(pl.tail) * pl.split * 256;
+    pl.ws_o = 0;
+    pl.ws_ml = align256(slots * d * sizeof(float));
+    pl.ws_bytes = pl.ws_ml + align256(slots * sizeof(float2));
+  }
+  return pl;
+}
+
 template <int D>
-safe_status launch_flash(FlashParams& p, cudaStream_t s) {
+safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t s) {
   constexpr int smem = flash_smem_bytes<D>();
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -113,16 +172,33 @@ safe_status launch_flash(FlashParams& p, cudaStream_t s) {
     attr_err = cudaFuncSetAttribute(flash_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
-  dim3 grid((p.n_q + 255) / 256, p.H, p.B);
+  FlashPlan pl = plan_flash(p.B, p.H, p.n_q, p.N, D, device_sms());
+  if (pl.split > 1 && (ws == nullptr || ws_bytes < pl.ws_bytes)) {
+    pl.full = pl.units;  // no workspace: whole units only
+    pl.split = 1;
+    pl.tail = 0;
+  }
+  p.n_mblk = (p.n_q + 255) / 256;
+  p.full_units = pl.full;
+  p.split = pl.split;
+  p.ws_o = nullptr;
+  p.ws_ml = nullptr;
+  if (pl.split > 1) {
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.ws_o = reinterpret_cast<float*>(w + pl.ws_o);
+    p.ws_ml = reinterpret_cast<float2*>(w + pl.ws_ml);
+  }
+  const unsigned grid = static_cast<unsigned>(pl.full + pl.tail * pl.split);
   flash_fwd_kernel<D><<<grid, kFlashThreads, smem, s>>>(p);
+  if (pl.split > 1) flash_merge_kernel<D><<<(pl.tail * 256 + 7) / 8, 256, 0, s>>>(p, pl.tail);
   return launch_status();
 }
 
-safe_status dispatch_flash(int d, FlashParams& p, cudaStream_t s) {
+safe_status dispatch_flash(int d, FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t s) {
   switch (d) {
-    case 64: return launch_flash<64>(p, s);
-    case 96: return launch_flash<96>(p, s);
-    case 128: return launch_flash<128>(p, s);
+    case 64: return launch_flash<64>(p, ws, ws_bytes, s);
+    case 96: return launch_flash<96>(p, ws, ws_bytes, s);
+    case 128: return launch_flash<128>(p, ws, ws_bytes, s);
     default: return SAFE_ERR_UNSUPPORTED;
   }
 }
@@ -282,8 +358,13 @@ safe_status safe_mask_classify_sync(const void* mask, int dtype, const int64_t s
   return cudaStreamSynchronize(s) == cudaSuccess ? SAFE_OK : SAFE_ERR_CUDA;
 }
 
+size_t safe_attn_workspace_bytes(int B, int n_q, int N, int H, int d) {
+  if (B < 1 || n_q < 1 || N < 1 || H < 1 || !supported_d(d)) return 0;
+  return plan_flash(B, H, n_q, N, d, device_sms()).ws_bytes;
+}
+
 safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O, float* lse, int B, int N, int H,
-                           int d, float scale, void* stream) {
+                           int d, float scale, void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SAFE_ERR_INVALID_ARG;
   if (!sizes_ok(B, N, H) || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
@@ -302,11 +383,12 @@ safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O,
   p.n_q = N;
   p.scale_log2 = scale * kLog2e;
   p.gather = 0;
-  return dispatch_flash(d, p, as_stream(stream));
+  return dispatch_flash(d, p, ws, ws_bytes, as_stream(stream));
 }
 
 safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
-                           void* O_S, float* lse, int B, int N, int H, int d, float scale, void* stream) {
+                           void* O_S, float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
+                           void* stream) {
   if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O_S)) return SAFE_ERR_INVALID_ARG;
   if (!sizes_ok(B, N, H) || k < 1 || k > N || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
   if (!q_compact && S == nullptr) return SAFE_ERR_INVALID_ARG;
@@ -328,7 +410,7 @@ safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k
   p.n_q = k;
   p.scale_log2 = scale * kLog2e;
   p.gather = q_compact ? 0 : 1;
-  return dispatch_flash(d, p, as_stream(stream));
+  return dispatch_flash(d, p, ws, ws_bytes, as_stream(stream));
 }
 
 safe_status safe_attn_cross(const void* Q, const int32_t* q_idx, int nq, const void* Ky, const void* Vy,

@@ -29,19 +29,21 @@ _SIGS = {
     "safe_abi_version": [],
     "safe_mask_classify": [_vp, _i, _i64p, _i64p, _vp, _vp],
     "safe_mask_classify_sync": [_vp, _i, _i64p, _i64p, _vp, _i64p, _vp],
-    "safe_attn_self": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp],
+    "safe_attn_workspace_bytes": [_i, _i, _i, _i, _i],
+    "safe_attn_self": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp],
     "safe_attn_cross": [_vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp],
     "safe_pcsp_workspace_bytes": [_i, _i, _i],
     "safe_pcsp_topk": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp],
     "safe_topk_partition": [_vp, _i, _i, _i, _vp, _vp, _vp],
-    "safe_srsu_attn": [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp],
+    "safe_srsu_attn": [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp],
     "safe_ctx_cache_scatter": [_vp, _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp],
     "safe_get_device_status": [ctypes.POINTER(ctypes.c_int), _vp],
     "safe_status_string": [_i],
     "safe_selftest_wait_timeout": [ctypes.c_uint64, _vp],
     "safe_pcsp_topk_noalloc": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
 }
-_RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_status_string": ctypes.c_char_p}
+_RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_attn_workspace_bytes": _sz,
+             "safe_status_string": ctypes.c_char_p}
 
 
 class SafeError(RuntimeError):
@@ -129,7 +131,24 @@ def _scale(d: int, scale: Optional[float]) -> float:
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
-def attn_self(Q, K, V, scale=None, return_lse=False, out=None, lse=None):
+def attn_workspace_bytes(B: int, n_q: int, N: int, H: int, d: int) -> int:
+    return int(lib().safe_attn_workspace_bytes(B, n_q, N, H, d))
+
+
+def _attn_ws(ws, B, n_q, N, H, d, device):
+    """Workspace for the wave-balancing key split: the given tensor, a fresh
+    one (ws=None), or no split at all (ws=False)."""
+    if ws is False:
+        return None, 0
+    if ws is None:
+        nbytes = attn_workspace_bytes(B, n_q, N, H, d)
+        if nbytes == 0:
+            return None, 0
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def attn_self(Q, K, V, scale=None, return_lse=False, out=None, lse=None, ws=None):
     """Mask-free image self-attention (Eq. (3) with the mask elided)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, n, torch.bfloat16, 4)
@@ -139,8 +158,9 @@ def attn_self(Q, K, V, scale=None, return_lse=False, out=None, lse=None):
     out = torch.empty_like(Q) if out is None else out
     if return_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    w, wb = _attn_ws(ws, B, N, N, H, d, Q.device)
     _check("safe_attn_self", lib().safe_attn_self(_p(Q), _p(K), _p(V), _p(out), _p(lse if return_lse else None),
-                                                  B, N, H, d, _scale(d, scale), _stream()))
+                                                  B, N, H, d, _scale(d, scale), _p(w), wb, _stream()))
     return (out, lse) if return_lse else out
 
 
@@ -210,7 +230,7 @@ def topk_partition(scores, k, S=None, C=None, with_c=True):
     return S, C
 
 
-def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=None, lse=None):
+def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=None, lse=None, ws=None):
     """SRSU selective self-attention (Eq. (16)): rows S of Q against all N
     keys of the assembled global K/V."""
     _need(Q, "Q", torch.bfloat16, 4)
@@ -222,9 +242,10 @@ def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=N
     out = torch.empty((B, k, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
     if return_lse and lse is None:
         lse = torch.empty((B, H, k), dtype=torch.float32, device=Q.device)
+    w, wb = _attn_ws(ws, B, k, N, H, d, Q.device)
     _check("safe_srsu_attn", lib().safe_srsu_attn(_p(Q), 1 if q_compact else 0, _p(S), k, _p(Kc), _p(Vc), _p(out),
                                                   _p(lse if return_lse else None), B, N, H, d, _scale(d, scale),
-                                                  _stream()))
+                                                  _p(w), wb, _stream()))
     return (out, lse) if return_lse else out
 
 

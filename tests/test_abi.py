@@ -47,10 +47,20 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.safe_abi_version() == 1
+    assert lib.safe_abi_version() == 2
     assert lib.safe_status_string(0) == b"ok"
     assert lib.safe_status_string(1) == b"invalid argument"
     assert lib.safe_status_string(99) == b"unknown status"
+
+
+def test_attn_workspace_plan(lib):
+    # wave-balancing workspace: needed when the last wave of 256-row units
+    # is partial, none when the units fill whole waves or keys are too few
+    lib.safe_attn_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.safe_attn_workspace_bytes(2, 6400, 25600, 24, 96) > 0      # 1200 units: 8.1 waves
+    assert lib.safe_attn_workspace_bytes(1, 256, 256, 2, 64) == 0         # 2 key tiles: no split
+    assert lib.safe_attn_workspace_bytes(0, 256, 256, 2, 64) == 0
+    assert lib.safe_attn_workspace_bytes(1, 256, 256, 2, 80) == 0
 
 
 def test_workspace_size(lib):
@@ -61,17 +71,17 @@ def test_workspace_size(lib):
 def test_host_validation_rejects_bad_arguments_without_gpu(lib):
     null = None
     # null / misaligned tensors, empty sizes, unsupported head dims
-    assert lib.safe_attn_self(null, null, null, null, null, 1, 1, 1, 96, 1.0, null) == 1
+    assert lib.safe_attn_self(null, null, null, null, null, 1, 1, 1, 96, 1.0, null, 0, null) == 1
     fake = ctypes.c_void_p(0x10000)
     odd = ctypes.c_void_p(0x10008)
-    assert lib.safe_attn_self(odd, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null) == 1
-    assert lib.safe_attn_self(fake, fake, fake, fake, null, 0, 16, 1, 96, 1.0, null) == 1
-    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 0, 1, 96, 1.0, null) == 1
-    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 80, 1.0, null) == 2
-    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 96, float("nan"), null) == 1
+    assert lib.safe_attn_self(odd, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 0, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 0, 1, 96, 1.0, null, 0, null) == 1
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 80, 1.0, null, 0, null) == 2
+    assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 96, float("nan"), null, 0, null) == 1
     # SRSU: k out of range
-    assert lib.safe_srsu_attn(fake, 0, fake, 0, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null) == 1
-    assert lib.safe_srsu_attn(fake, 0, fake, 17, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null) == 1
+    assert lib.safe_srsu_attn(fake, 0, fake, 0, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert lib.safe_srsu_attn(fake, 0, fake, 17, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
     # cross: M > 256 unsupported, nq must equal N without q_idx
     assert lib.safe_attn_cross(fake, null, 16, fake, fake, fake, fake, 1, 16, 257, 1, 96, 1.0, null) == 2
     assert lib.safe_attn_cross(fake, null, 8, fake, fake, fake, fake, 1, 16, 16, 1, 96, 1.0, null) == 1

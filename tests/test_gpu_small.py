@@ -361,6 +361,37 @@ def test_srsu_bad_index_flagged():
     assert ops.device_status() & (1 << ops.SAFE_ERR_DEVICE_CHECK)
 
 
+@pytest.mark.parametrize("B,N,H,d,k", [(1, 4096, 2, 96, 4096), (2, 3000, 3, 64, 1500), (1, 4096, 1, 128, 777),
+                                       (2, 4096, 3, 96, 1229)])
+def test_key_split_wave_balancing_matches_oracle(B, N, H, d, k):
+    # the last partial wave of CTAs is split along the keys and merged by
+    # the last part; the workspace needs no initialisation (filled with NaN)
+    Q, K, V = rand_qkv(B, N, H, d, seed=N + 3 * k)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    nbytes = ops.attn_workspace_bytes(B, k, N, H, d)
+    assert nbytes > 0
+    ws = torch.full((nbytes // 4,), float("nan"), dtype=torch.float32, device=DEV).view(torch.uint8)
+    scale = 1 / math.sqrt(d)
+    if k == N:
+        out, lse = ops.attn_self(Qd, Kd, Vd, return_lse=True, ws=ws)
+        out_whole, lse_whole = ops.attn_self(Qd, Kd, Vd, return_lse=True, ws=False)
+        ref, ref_lse = O.attention(to64(Q), to64(K), to64(V), scale, with_lse=True)
+    else:
+        S = np.stack([np.sort(np.random.default_rng(b + 5).choice(N, k, replace=False)) for b in range(B)])
+        Sd = torch.from_numpy(S.astype(np.int32)).to(DEV)
+        out, lse = ops.srsu_attn(Qd, Sd, Kd, Vd, return_lse=True, ws=ws)
+        out_whole, lse_whole = ops.srsu_attn(Qd, Sd, Kd, Vd, return_lse=True, ws=False)
+        ref, ref_lse = O.attention(to64(Q), to64(K), to64(V), scale, q_rows=S, with_lse=True)
+    assert_attn_close(out, ref, "split")
+    assert_attn_close(out_whole, ref, "whole")
+    np.testing.assert_allclose(to64(lse), ref_lse, atol=2e-3, rtol=0)
+    np.testing.assert_allclose(to64(lse_whole), ref_lse, atol=2e-3, rtol=0)
+    # a second call reuses the workspace
+    out2 = ops.attn_self(Qd, Kd, Vd, ws=ws) if k == N else ops.srsu_attn(Qd, Sd, Kd, Vd, ws=ws)
+    assert torch.equal(out2, out)
+    assert ops.device_status() == 0
+
+
 # ---------------------------------------------------------------- failure detection
 
 
