@@ -42,6 +42,22 @@ WORKLOAD = "2560^2-equivalent SRSU step: B=2, H=24, d=96, N=25600, M=128 (len U[
 LAUNCHES_PER_STEP = 11
 
 
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """Largest per-rank device time (ms): the job is as slow as its slowest
+    rank. Identity for a single process."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own replica of the step (weak
+    scaling), so the job does world x the work of one rank per step time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -383,13 +399,9 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    ms_total = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     ms_step = ms_total / args.steps
-    value = world * f_step / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, f_step, ms_step)
 
     # end to end through the public API with host buffers: H2D of the step's
     # inputs from pinned memory, the step, D2H of its outputs
@@ -409,12 +421,8 @@ def main():
             ho.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1) / e_steps
-    if dist is not None:
-        tt = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
-    e2e = {"value": world * f_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / e_steps, dist, dev)
+    e2e = {"value": job_throughput(world, f_step, ms_e2e), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     dense_list, srsu_list = step.launch_times()
