@@ -212,7 +212,13 @@ safe_status launch_cross(CrossParams& p, cudaStream_t s) {
     attr_err = cudaFuncSetAttribute(cross_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
-  dim3 grid((p.nq + 127) / 128, p.H, p.B);
+  // a few CTAs per (b, h), each streaming a contiguous range of query tiles,
+  // all resident at once: two CTAs per SM (one for M > 128)
+  const int n_tiles = (p.nq + 127) / 128;
+  const int resident = device_sms() * (p.M <= 128 ? 2 : 1);
+  int per_bh = resident / (p.B * p.H);
+  per_bh = per_bh < 1 ? 1 : (per_bh > n_tiles ? n_tiles : per_bh);
+  dim3 grid(per_bh, p.H, p.B);
   cross_attn_kernel<D><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
   return launch_status();
 }
