@@ -3,21 +3,29 @@
 // partial scores built from the same probabilities (Eq. (9), (10)).
 //
 // All M <= 256 text keys of a (b, h) fit one tile, so the softmax is exact in
-// one pass over them. A few CTAs (4 warps each) share the query tiles of one
-// (b, h); each CTA
-//   1. copies the first Lp = ceil32(valid_len) text key / value rows into the
-//      swizzled shared-memory layout the tensor core reads, once, writing
-//      zeros for rows >= valid_len (padding rows are never read, so they may
-//      hold any bytes), with all of a thread's loads in flight together;
-//   2. streams its range of 128-row query tiles through a two-buffer TMA
-//      ring (dense rows, or rows of S via gather4), the next tile's load in
-//      flight while the current one is processed;
-//   3. per tile: S = Q Ky^T (M=128, N=Lp) into TMEM; each thread owns one
-//      query row: max over valid keys, p = 2^(s*scale*log2(e) - max),
-//      l = sum p, score = sum_j w_j p_j / l (the PCSP partial for this head);
-//      P (bf16) goes back into TMEM and O = P Vy / l is written as bf16.
-// Two CTAs fit an SM (M <= 128), so one CTA's softmax overlaps the other's
-// loads and MMAs.
+// one pass over them. A CTA (one per SM) owns a range of 128-row query tiles
+// of one (b, h) and pipelines them:
+//   warp 0      TMA producer: query tiles (dense rows, or rows of S via
+//               gather4) into a ring of QS shared-memory slots;
+//   warps 1, 2  MMA issuers, one per softmax warpgroup (even / odd tiles):
+//               S = Q Ky^T (N = Lp = ceil32(valid_len)) into TMEM, then
+//               O = P Vy with P read from TMEM;
+//   warp 3      output store: the bf16 O tile, staged by the warpgroup in
+//               the slot its query tile came from, leaves by TMA store, and
+//               the slot returns to the producer;
+//   warps 4..11 two softmax warpgroups, one query row per thread: max over
+//               the valid keys, p = 2^(s*scale*log2(e) - max), l = sum p,
+//               score = sum_j w_j p_j / l (the PCSP partial of this head),
+//               P (bf16) back into TMEM; after P V, O / l into the slot.
+// Before the first tile the text key / value rows [0, Lp) are copied into the
+// swizzled layouts the tensor core reads, zeros for rows >= valid_len
+// (padding rows are never read, so they may hold any bytes).
+//
+// TMEM (512 columns): warpgroup g owns [256g, 256g + 256): S in [0, Lp), P
+// (bf16 pairs) over its first Lp/2 columns, O in [128, 128 + D). For
+// Lp <= 128 the next S of a warpgroup only waits for the previous P V
+// product; for Lp > 128 it overlaps O and waits for the previous output to
+// be read.
 #pragma once
 
 #include "flash_attn.cuh"
@@ -27,6 +35,7 @@ namespace safe {
 struct CrossParams {
   CUtensorMap q_map[2];   // 4-D dense Q map per chunk
   CUtensorMap qg_map[2];  // 2-D gather map per chunk
+  CUtensorMap o_map[2];   // 4-D map of O [B, nq, H, D] per chunk (stores)
   const __nv_bfloat16* Ky;  // [B, M, H, D]
   const __nv_bfloat16* Vy;
   const int32_t* valid_len;  // [B]
@@ -37,35 +46,52 @@ struct CrossParams {
   int B, N, M, H, nq;
   float scale_log2;
   int gather;
+  int qs;  // query-tile slots in shared memory
 };
 
-constexpr int kCrossThreads = 128;
+constexpr int kCrossThreads = 384;
+constexpr int kCrossMaxSmem = 232448 - 1024;  // dynamic shared memory limit of one CTA, less room for the static part
+constexpr int kCrossMinSmem = 120 * 1024;  // keeps the CTA alone on its SM (it holds all of TMEM)
 
+template <int D>
+__host__ __device__ constexpr int cross_smem_need(int M, int qs) {
+  return 1024 + qs * TileCfg<D>::kTileBytes + 2 * (((M + 31) / 32) * 32) * D * 2 + 256 * 4 + 256;
+}
+// Slots that fit next to the text keys / values (4 at most, 2 at least).
+template <int D>
+__host__ __device__ constexpr int cross_slots(int M) {
+  return cross_smem_need<D>(M, 4) <= kCrossMaxSmem ? 4 : (cross_smem_need<D>(M, 3) <= kCrossMaxSmem ? 3 : 2);
+}
 template <int D>
 __host__ __device__ constexpr int cross_smem_bytes(int M) {
-  return 1024 + 2 * TileCfg<D>::kTileBytes + 2 * (((M + 31) / 32) * 32) * D * 2 + 256 * 4 + 64;
-}
-
-__host__ __device__ constexpr int cross_tmem_cols(int M, int D) {
-  return ((M <= 128 ? 128 : 256) + D) <= 256 ? 256 : 512;
+  return cross_smem_need<D>(M, cross_slots<D>(M)) < kCrossMinSmem ? kCrossMinSmem
+                                                                  : cross_smem_need<D>(M, cross_slots<D>(M));
 }
 
 template <int D>
-__global__ void __launch_bounds__(kCrossThreads) cross_attn_kernel(const __grid_constant__ CrossParams p) {
+__global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __grid_constant__ CrossParams p) {
   using C = TileCfg<D>;
   constexpr int TB = C::kTileBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int QS = p.qs;
   const int Mp = ((p.M + 31) / 32) * 32;
-  uint8_t* sQ = sm;  // two query-tile buffers
-  uint8_t* sKy = sQ + 2 * TB;
+  uint8_t* sQ = sm;  // QS query-tile slots (also the output staging)
+  uint8_t* sKy = sQ + QS * TB;
   uint8_t* sVy = sKy + Mp * D * 2;
   float* sw = reinterpret_cast<float*>(sVy + Mp * D * 2);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sw + 256);
-  uint64_t* q_full = bars;      // [2]
-  uint64_t* s_bar = bars + 2;
-  uint64_t* o_bar = bars + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* q_full = bars;         // [4]
+  uint64_t* q_empty = bars + 4;    // [4]
+  uint64_t* s_full = bars + 8;     // [2] per warpgroup
+  uint64_t* p_full = bars + 10;    // [2]
+  uint64_t* o_full = bars + 12;    // [2]
+  uint64_t* t_free = bars + 14;    // [2] TMEM S / O of the warpgroup read
+  // [4] output tile written to its slot (per slot: a slot's next output
+  // waits for this one's store, so its phases are never skipped)
+  uint64_t* o_staged = bars + 16;
+  uint64_t* drained = bars + 20;  // [2] issuer's MMAs all complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -76,8 +102,7 @@ __global__ void __launch_bounds__(kCrossThreads) cross_attn_kernel(const __grid_
   const int tile1 = tile0 + per < n_tiles ? tile0 + per : n_tiles;
   if (tile0 >= tile1) return;  // uniform for the CTA, before any barrier or TMEM use
   const int n_my = tile1 - tile0;
-  const int s_region = p.M <= 128 ? 128 : 256;
-  const uint32_t tcols = static_cast<uint32_t>(cross_tmem_cols(p.M, D));
+  const bool has_o = p.O != nullptr;
 
   int L = __ldg(p.valid_len + b);
   if (L < 1 || L > p.M) {
@@ -88,30 +113,36 @@ __global__ void __launch_bounds__(kCrossThreads) cross_attn_kernel(const __grid_
 
   if (tid == 0) {
     abort_flag = 0;
-    mbar_init(&q_full[0], 1);
-    mbar_init(&q_full[1], 1);
-    mbar_init(s_bar, 1);
-    mbar_init(o_bar, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&o_staged[i], 128);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&p_full[g], 128);
+      mbar_init(&o_full[g], 1);
+      mbar_init(&t_free[g], 128);
+      mbar_init(&drained[g], 1);
+    }
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, tcols);
+  if (warp == 0) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  // query tile `it` of this CTA -> buffer it & 1 (issued by warp 0)
-  int q_issued = 0;
+  // query tile `it` of this CTA -> slot it % QS (issued by the whole warp 0)
   auto load_q = [&](int it) {
-    const int buf = it & 1;
-    q_issued = it + 1;
+    const int slot = it % QS;
+    uint8_t* dst = sQ + slot * TB;
     const int q0 = (tile0 + it) * 128;
-    if (lane == 0) mbar_arrive_expect_tx(&q_full[buf], TB);
+    if (lane == 0) mbar_arrive_expect_tx(&q_full[slot], TB);
     __syncwarp();
     if (!p.gather) {
       if (lane == 0)
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sQ + buf * TB + C::chunk_off(c), &p.q_map[c], &q_full[buf], 64 * c, h, q0, b);
+        for (int c = 0; c < C::kChunks; ++c) tma_load_4d(dst + C::chunk_off(c), &p.q_map[c], &q_full[slot], 64 * c, h, q0, b);
     } else {
       int y[4];
       for (int u = 0; u < 4; ++u) {
@@ -125,39 +156,39 @@ __global__ void __launch_bounds__(kCrossThreads) cross_attn_kernel(const __grid_
         y[u] = b * p.N + idx;
       }
       for (int c = 0; c < C::kChunks; ++c)
-        tma_gather4(sQ + buf * TB + C::chunk_off(c) + 4 * lane * C::row_bytes(c), &p.qg_map[c], &q_full[buf],
+        tma_gather4(dst + C::chunk_off(c) + 4 * lane * C::row_bytes(c), &p.qg_map[c], &q_full[slot],
                     h * D + 64 * c, y[0], y[1], y[2], y[3]);
     }
   };
+  int q_issued = 0;
   if (warp == 0) {
-    load_q(0);
-    if (n_my > 1) load_q(1);
-  }
-
-  // text keys / values -> swizzled shared memory (zeros past valid_len);
-  // eight 16-byte units per thread are loaded before any is stored
-  {
+    for (; q_issued < n_my && q_issued < QS; ++q_issued) load_q(q_issued);
+  } else if (warp >= 3) {
+    // text keys / values -> swizzled shared memory (zeros past valid_len);
+    // eight 16-byte units per thread are loaded before any is stored
     constexpr int kUnits = D / 8;  // 16-byte units per row
+    constexpr int kCopyThreads = kCrossThreads - 96;
+    const int ct = tid - 96;
     const size_t row_stride = static_cast<size_t>(p.H) * D;  // elements between text tokens
     const __nv_bfloat16* kbase = p.Ky + (static_cast<size_t>(b) * p.M * p.H + h) * D;
     const __nv_bfloat16* vbase = p.Vy + (static_cast<size_t>(b) * p.M * p.H + h) * D;
     const int total = Lp * kUnits;
-    for (int e0 = tid; e0 < total; e0 += 8 * kCrossThreads) {
+    for (int e0 = ct; e0 < total; e0 += 8 * kCopyThreads) {
       uint4 kv[8], vv[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int e = e0 + k * kCrossThreads;
+        const int e = e0 + k * kCopyThreads;
         const int r = e / kUnits, u = e % kUnits;
         kv[k] = make_uint4(0, 0, 0, 0);
         vv[k] = make_uint4(0, 0, 0, 0);
         if (e < total && r < L) {
           kv[k] = __ldg(reinterpret_cast<const uint4*>(kbase + r * row_stride) + u);
-          if (p.O != nullptr) vv[k] = __ldg(reinterpret_cast<const uint4*>(vbase + r * row_stride) + u);
+          if (has_o) vv[k] = __ldg(reinterpret_cast<const uint4*>(vbase + r * row_stride) + u);
         }
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int e = e0 + k * kCrossThreads;
+        const int e = e0 + k * kCopyThreads;
         if (e >= total) break;
         const int r = e / kUnits, u = e % kUnits;
         // K (K-major operand): 64-wide chunks, 128B swizzle (+ a 32-wide,
@@ -173,186 +204,245 @@ __global__ void __launch_bounds__(kCrossThreads) cross_attn_kernel(const __grid_
             vv[k];
       }
     }
-    for (int j = tid; j < Lp; j += kCrossThreads) {
+    for (int j = ct; j < Lp; j += kCopyThreads) {
       float wj = 0.f;
       if (j < L) wj = p.w != nullptr ? __ldg(p.w + static_cast<size_t>(b) * p.M + j) : 1.f / static_cast<float>(L);
       sw[j] = wj;
     }
+    fence_proxy_async_smem();
   }
-  fence_proxy_async_smem();
   __syncthreads();
 
-  const int quarter = warp & 3;
-  const int row = quarter * 32 + lane;
-  const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t tS = tbase + lane_addr;
-  const uint32_t tO = tbase + lane_addr + s_region;
-  const float sl2 = p.scale_log2;
-  const uint32_t idS = make_idesc_bf16(128, Lp, 0, 0);
-  constexpr uint32_t idPV = make_idesc_bf16(128, D, 0, 1);
-  const uint32_t aK = smem_u32(sKy), aV = smem_u32(sVy);
-
-  bool ok = true;
-  for (int it = 0; it < n_my && ok; ++it) {
-    const int buf = it & 1;
-    const int q_row = (tile0 + it) * 128 + row;
-    const bool valid = q_row < p.nq;
-    // S = Q Ky^T
-    if (tid == 0) {
-      if (mbar_wait(&q_full[buf], (it >> 1) & 1, &abort_flag)) {
+  if (warp < 4) {
+  regs_dealloc<kRegsControl>();  // (warpgroup-wide, as is the increase below)
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    bool ok = true;
+    for (; q_issued < n_my; ++q_issued) {
+      const int slot = q_issued % QS;
+      ok = warp_wait(&q_empty[slot], ((q_issued / QS) - 1) & 1, &abort_flag);
+      if (!ok) break;
+      load_q(q_issued);
+    }
+    if (lane == 0) {
+      // the loads this CTA started have landed before it exits (already
+      // true unless another role gave up)
+      for (int i = q_issued - QS < 0 ? 0 : q_issued - QS; i < q_issued; ++i)
+        mbar_wait_drain(&q_full[i % QS], (i / QS) & 1);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    const int g = warp - 1;
+    if (lane == 0) {
+      const uint32_t tS = tbase + 256 * g, tO = tS + 128;
+      const uint32_t idS = make_idesc_bf16(128, Lp, 0, 0);
+      constexpr uint32_t idPV = make_idesc_bf16(128, D, 0, 1);
+      const uint32_t aK = smem_u32(sKy), aV = smem_u32(sVy);
+      for (int i = g; i < n_my; i += 2) {
+        const int k = i >> 1, slot = i % QS;
+        if (!mbar_wait(&q_full[slot], (i / QS) & 1, &abort_flag)) break;
+        // the previous tile of this warpgroup has released S (and, when S
+        // reaches into the O columns, its output)
+        if (k > 0) {
+          uint64_t* prev = (has_o && Lp <= 128) ? &o_full[g] : &t_free[g];
+          if (!mbar_wait(prev, (k - 1) & 1, &abort_flag)) break;
+        }
         tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ + buf * TB);
+        const uint32_t aQ = smem_u32(sQ + slot * TB);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2;
           const uint64_t bd = make_sdesc(aK + c * Mp * 128 + (kk & 3) * 32, 16, 8 * C::row_bytes(c), C::swizzle(c));
-          umma_ss(tbase, kmajor_desc<D>(aQ, kk), bd, idS, kk > 0 ? 1u : 0u);
+          umma_ss(tS, kmajor_desc<D>(aQ, kk), bd, idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(s_bar);
-      }
-    }
-    // (bounded waits; the outcome is made CTA-uniform before going on)
-    ok = __syncthreads_and(mbar_wait(s_bar, it & 1, &abort_flag));
-    if (!ok) break;
-    tc_fence_after();
-    // the S product has read Q buffer `buf`: refill it with tile it + 2
-    if (warp == 0 && it + 2 < n_my) load_q(it + 2);
-    float l = 0.f, score = 0.f;
-    if (Lp <= 128) {
-      // all of S in registers: one TMEM pass. Only the last 32-key chunk can
-      // hold padding keys; they are set to -inf (their weights are 0).
-      uint32_t sr[128];
-      const int nc = Lp / 32;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < nc) tmem_ld32(tS + 32 * c, sr + 32 * c);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < nc) tmem_ld_wait32(sr + 32 * c);  // ties the loaded registers to the wait
-#pragma unroll
-      for (int j = 0; j < 128; ++j)
-        if (j >= L) sr[j] = __float_as_uint(-INFINITY);
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c < nc) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              m4[k] = fmax3(m4[k], __uint_as_float(sr[32 * c + i + 2 * k]), __uint_as_float(sr[32 * c + i + 2 * k + 1]));
+        umma_commit(&s_full[g]);
+        if (!has_o) {
+          umma_commit(&q_empty[slot]);
+          continue;
         }
-      }
-      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), neg2 = f2_pack(-mx * sl2, -mx * sl2);
-      uint64_t lacc[2] = {0, 0}, sacc[2] = {0, 0};  // packed row sums and weighted sums
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c >= nc) continue;
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j0 = 32 * c + 2 * i;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), sl2x2, neg2), x0, x1);
-          const float a = ex2_approx(x0), bb = ex2_approx(x1);
-          const uint64_t e2 = f2_pack(a, bb);
-          const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
-          lacc[i & 1] = f2_add(lacc[i & 1], e2);
-          sacc[i & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i & 1]);
-          pk[i] = pack_bf16x2(a, bb);
-        }
-        if (p.O != nullptr) tmem_st16(tS + 16 * c, pk);
-      }
-      float l0, l1, l2, l3, s0, s1, s2, s3;
-      f2_unpack(lacc[0], l0, l1);
-      f2_unpack(lacc[1], l2, l3);
-      f2_unpack(sacc[0], s0, s1);
-      f2_unpack(sacc[1], s2, s3);
-      l = (l0 + l1) + (l2 + l3);
-      score = (s0 + s1) + (s2 + s3);
-    } else {
-      // pass 1: row max over valid keys
-      float mx = -INFINITY;
-      for (int c = 0; c < Lp / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tS + 32 * c, sr);
-        tmem_ld_wait32(sr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (32 * c + i < L) mx = fmaxf(mx, __uint_as_float(sr[i]));
-      }
-      const float neg = -mx * sl2;
-      // pass 2: probabilities, sums, P -> TMEM
-      for (int c = 0; c < Lp / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tS + 32 * c, sr);
-        tmem_ld_wait32(sr);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j0 = 32 * c + 2 * i;
-          const float a = j0 < L ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, neg)) : 0.f;
-          const float bb = j0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, neg)) : 0.f;
-          l += a + bb;
-          score = fmaf(sw[j0], a, score);
-          score = fmaf(sw[j0 + 1], bb, score);
-          pk[i] = pack_bf16x2(a, bb);
-        }
-        if (p.O != nullptr) tmem_st16(tS + 16 * c, pk);
-      }
-    }
-    if (p.partial != nullptr && valid)
-      p.partial[(static_cast<size_t>(b) * p.H + h) * p.nq + q_row] = score / l;
-
-    if (p.O != nullptr) {
-      // O = P Vy / l
-      tmem_st_wait();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0 && !abort_flag) {
+        if (!mbar_wait(&p_full[g], k & 1, &abort_flag)) break;
+        if (k > 0 && !mbar_wait(&t_free[g], (k - 1) & 1, &abort_flag)) break;
         tc_fence_after();
         for (int kk = 0; kk < Lp / 16; ++kk)
-          umma_ts(tbase + s_region, tbase + kk * 8, make_sdesc(aV + kk * 16 * 64, Mp * 64, 512, kSwizzle64B), idPV,
-                  kk > 0 ? 1u : 0u);
-        umma_commit(o_bar);
+          umma_ts(tO, tS + kk * 8, make_sdesc(aV + kk * 16 * 64, Mp * 64, 512, kSwizzle64B), idPV, kk > 0 ? 1u : 0u);
+        umma_commit(&o_full[g]);
       }
-      ok = __syncthreads_and(mbar_wait(o_bar, it & 1, &abort_flag));
-      if (!ok) break;
+      // every MMA this thread issued has completed before TMEM is released
+      umma_commit(&drained[g]);
+      mbar_wait_drain(&drained[g], 0);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ output store
+    if (has_o && lane == 0) {
+      for (int i = 0; i < n_my; ++i) {
+        const int slot = i % QS;
+        if (!mbar_wait(&o_staged[slot], (i / QS) & 1, &abort_flag)) break;
+        const uint8_t* src = sQ + slot * TB;
+        const int q0 = (tile0 + i) * 128;
+        for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&p.o_map[c], src + C::chunk_off(c), 64 * c, h, q0, b);
+        bulk_commit_group();
+        bulk_wait_read_all();
+        mbar_arrive(&q_empty[slot]);
+      }
+      bulk_wait_all();
+    }
+  }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    regs_alloc<kRegsSoftmax>();
+    const int g = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tbase + 256 * g + lane_addr;
+    const uint32_t tO = tS + 128;
+    const float sl2 = p.scale_log2;
+    for (int i = g; i < n_my; i += 2) {
+      const int k = i >> 1;
+      const int q_row = (tile0 + i) * 128 + row;
+      const bool valid = q_row < p.nq;
+      if (!warp_wait(&s_full[g], k & 1, &abort_flag)) break;
+      tc_fence_after();
+      float l = 0.f, score = 0.f;
+      if (Lp <= 128) {
+        // all of S in registers: one TMEM pass. Only the last 32-key chunk
+        // can hold padding keys; they are set to -inf (their weights are 0).
+        uint32_t sr[128];
+        const int nc = Lp / 32;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < nc) tmem_ld32(tS + 32 * c, sr + 32 * c);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < nc) tmem_ld_wait32(sr + 32 * c);  // ties the loaded registers to the wait
+        if (!has_o) {
+          tc_fence_before();
+          mbar_arrive(&t_free[g]);
+        }
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (j >= L) sr[j] = __float_as_uint(-INFINITY);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c < nc) {
+#pragma unroll
+            for (int i2 = 0; i2 < 32; i2 += 8)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                m4[q] = fmax3(m4[q], __uint_as_float(sr[32 * c + i2 + 2 * q]), __uint_as_float(sr[32 * c + i2 + 2 * q + 1]));
+          }
+        }
+        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), neg2 = f2_pack(-mx * sl2, -mx * sl2);
+        uint64_t lacc[2] = {0, 0}, sacc[2] = {0, 0};  // packed row sums and weighted sums
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c >= nc) continue;
+          uint32_t pk[16];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const int j0 = 32 * c + 2 * i2;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), sl2x2, neg2), x0, x1);
+            const float a = ex2_approx(x0), bb = ex2_approx(x1);
+            const uint64_t e2 = f2_pack(a, bb);
+            const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
+            lacc[i2 & 1] = f2_add(lacc[i2 & 1], e2);
+            sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+            pk[i2] = pack_bf16x2(a, bb);
+          }
+          if (has_o) tmem_st16(tS + 16 * c, pk);
+        }
+        float l0, l1, l2, l3, s0, s1, s2, s3;
+        f2_unpack(lacc[0], l0, l1);
+        f2_unpack(lacc[1], l2, l3);
+        f2_unpack(sacc[0], s0, s1);
+        f2_unpack(sacc[1], s2, s3);
+        l = (l0 + l1) + (l2 + l3);
+        score = (s0 + s1) + (s2 + s3);
+      } else {
+        // pass 1: row max over valid keys
+        float mx = -INFINITY;
+        for (int c = 0; c < Lp / 32; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tS + 32 * c, sr);
+          tmem_ld_wait32(sr);
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2)
+            if (32 * c + i2 < L) mx = fmaxf(mx, __uint_as_float(sr[i2]));
+        }
+        const float neg = -mx * sl2;
+        // pass 2: probabilities, sums, P -> TMEM (P chunk c lands on S
+        // columns already read)
+        for (int c = 0; c < Lp / 32; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tS + 32 * c, sr);
+          tmem_ld_wait32(sr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const int j0 = 32 * c + 2 * i2;
+            const float a = j0 < L ? ex2_approx(fmaf(__uint_as_float(sr[2 * i2]), sl2, neg)) : 0.f;
+            const float bb = j0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(sr[2 * i2 + 1]), sl2, neg)) : 0.f;
+            l += a + bb;
+            score = fmaf(sw[j0], a, score);
+            score = fmaf(sw[j0 + 1], bb, score);
+            pk[i2] = pack_bf16x2(a, bb);
+          }
+          if (has_o) tmem_st16(tS + 16 * c, pk);
+        }
+        if (!has_o) {
+          tc_fence_before();
+          mbar_arrive(&t_free[g]);
+        }
+      }
+      if (has_o) {
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[g]);
+      }
+      if (p.partial != nullptr && valid) p.partial[(static_cast<size_t>(b) * p.H + h) * p.nq + q_row] = score / l;
+      if (!has_o) continue;
+
+      // O = P Vy / l -> bf16 into the slot of this tile's queries (the S
+      // product has read them), laid out like a query tile for the store
+      if (!warp_wait(&o_full[g], k & 1, &abort_flag)) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.nq + (valid ? q_row : 0)) * p.H + h) * D;
+      uint8_t* slot = sQ + (i % QS) * TB;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
         tmem_ld_wait32(o);
+        if (c == D / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&t_free[g]);
+        }
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        for (int i2 = 0; i2 < 16; ++i2)
+          pk[i2] = pack_bf16x2(__uint_as_float(o[2 * i2]) * inv_l, __uint_as_float(o[2 * i2 + 1]) * inv_l);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int v = 0; v < 4; ++v) {
+          const int u = 4 * c + v;  // 16-byte unit of the row
+          const int cq = u >> 3, uc = u & 7;
+          const int rb = C::row_bytes(cq);
+          const int xr = (rb == 128) ? (row & 7) : ((row >> 1) & 3);
+          *reinterpret_cast<uint4*>(slot + C::chunk_off(cq) + row * rb + ((uc ^ xr) << 4)) =
+              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&o_staged[i % QS]);
     }
-    // every thread has read S / O of this tile before the next S overwrites them
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
-  if (!ok && warp == 0) {
-    // let the query loads this CTA started land before it exits
-    for (int i = q_issued - 2 < 0 ? 0 : q_issued - 2; i < q_issued; ++i)
-      mbar_wait_drain(&q_full[i & 1], (i >> 1) & 1);
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tbase, tcols);
+  if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
 // scores[b, i] (+)= (1/H) * sum_h partial[b, h, i], heads summed in order.

@@ -205,19 +205,18 @@ safe_status dispatch_flash(int d, FlashParams& p, void* ws, size_t ws_bytes, cud
 
 template <int D>
 safe_status launch_cross(CrossParams& p, cudaStream_t s) {
-  const int smem = cross_smem_bytes<D>(256);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [smem] {
-    attr_err = cudaFuncSetAttribute(cross_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(cross_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kCrossMaxSmem);
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
-  // a few CTAs per (b, h), each streaming a contiguous range of query tiles,
-  // all resident at once: two CTAs per SM (one for M > 128)
+  // one CTA per SM (each holds all of TMEM), a few per (b, h), each streaming
+  // a contiguous range of query tiles
   const int n_tiles = (p.nq + 127) / 128;
-  const int resident = device_sms() * (p.M <= 128 ? 2 : 1);
-  int per_bh = resident / (p.B * p.H);
+  int per_bh = device_sms() / (p.B * p.H);
   per_bh = per_bh < 1 ? 1 : (per_bh > n_tiles ? n_tiles : per_bh);
+  p.qs = cross_slots<D>(p.M);
   dim3 grid(per_bh, p.H, p.B);
   cross_attn_kernel<D><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
   return launch_status();
@@ -249,6 +248,9 @@ safe_status fill_cross(CrossParams& p, const void* Q, const int32_t* q_idx, int 
       if (!encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c)) return SAFE_ERR_CUDA;
     }
   }
+  if (O != nullptr)
+    for (int c = 0; c < nchunks(d); ++c)
+      if (!encode_rows_map(&p.o_map[c], O, B, nq, H, d, c)) return SAFE_ERR_CUDA;
   p.Ky = static_cast<const __nv_bfloat16*>(Ky);
   p.Vy = static_cast<const __nv_bfloat16*>(Vy);
   p.valid_len = valid_len;

@@ -187,6 +187,44 @@ def test_attn_cross_row_selection_equals_dense_rows():
     assert_attn_close(sel, ref, "cross rows")
 
 
+# More (b, h) pairs than SMs: one CTA per (b, h) streams every query tile of
+# its head, so the query-slot ring wraps several times and both softmax
+# warpgroups see several tiles (odd and even counts, both softmax forms).
+@pytest.mark.parametrize("B,N,M,H,d,lens,rows", [(2, 2000, 128, 80, 96, [77, 128], None),
+                                                 (1, 1700, 256, 150, 128, [200], None),
+                                                 (2, 3000, 128, 80, 64, [5, 96], 1500),
+                                                 (1, 2200, 40, 160, 96, [33], 1111)])
+def test_attn_cross_many_tiles_per_cta(B, N, M, H, d, lens, rows):
+    Q = rnd_bf16((B, N, H, d), 71)
+    Ky, Vy = rnd_bf16((B, M, H, d), 72), rnd_bf16((B, M, H, d), 73)
+    L = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    S = None
+    if rows is not None:
+        S = torch.stack([torch.from_numpy(np.sort(np.random.default_rng(70 + b).choice(N, rows, replace=False)))
+                         for b in range(B)]).to(torch.int32)
+    out = ops.attn_cross(Q.to(DEV), Ky.to(DEV), Vy.to(DEV), L, q_idx=None if S is None else S.to(DEV))
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0  # no wait of the pipeline ran out
+    ref = O.cross_attention(to64(Q), to64(Ky), to64(Vy), lens, 1 / math.sqrt(d),
+                            q_rows=None if S is None else S.numpy())
+    # valid lengths down to 5 keys give output rows of magnitude up to ~4,
+    # where one bf16 rounding step of the output alone is ~1e-2
+    assert_attn_close(out, ref, "cross many tiles", magnitude_scaled=True)
+
+
+def test_pcsp_scores_many_tiles_per_cta():
+    B, N, M, H, d = 2, 2000, 128, 80, 96
+    Q = rnd_bf16((B, N, H, d), 81)
+    Ky = rnd_bf16((B, M, H, d), 82)
+    lens = [100, 17]
+    w = synth.content_weights(torch.tensor(lens), M, 83)
+    sc, _, _ = ops.pcsp_topk(Q.to(DEV), Ky.to(DEV), torch.tensor(lens, dtype=torch.int32, device=DEV), w.to(DEV))
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    ref = O.pcsp_scores(to64(Q), to64(Ky), lens, w.numpy().astype(np.float64), 1 / math.sqrt(d))
+    np.testing.assert_allclose(sc.cpu().numpy(), ref, rtol=2e-5, atol=1e-8)
+
+
 def test_attn_cross_invalid_length_is_flagged_not_faulted():
     Q = rnd_bf16((1, 128, 1, 64), 1).to(DEV)
     Ky = rnd_bf16((1, 16, 1, 64), 2).to(DEV)
