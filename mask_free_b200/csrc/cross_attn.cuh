@@ -19,7 +19,11 @@
 //               P (bf16) back into TMEM; after P V, O / l into the slot.
 // Before the first tile the text key / value rows [0, Lp) are copied into the
 // swizzled layouts the tensor core reads, zeros for rows >= valid_len
-// (padding rows are never read, so they may hold any bytes).
+// (padding rows are never read, so they may hold any bytes). The padding
+// keys are masked by the tensor core itself: one more K = 16 step adds
+// ones(128 x 16) . bias(Lp x 16)^T to S, with bias rows 0 for valid keys and
+// -inf for padding keys, so S arrives with -inf in every padding column and
+// the softmax has no mask to apply.
 //
 // TMEM (512 columns): warpgroup g owns [256g, 256g + 256): S in [0, Lp), P
 // (bf16 pairs) over its first Lp/2 columns, O in [128, 128 + D). For
@@ -27,6 +31,8 @@
 // product; for Lp > 128 it overlaps O and waits for the previous output to
 // be read.
 #pragma once
+
+#include <type_traits>
 
 #include "flash_attn.cuh"
 
@@ -53,9 +59,22 @@ constexpr int kCrossThreads = 384;
 constexpr int kCrossMaxSmem = 232448 - 1024;  // dynamic shared memory limit of one CTA, less room for the static part
 constexpr int kCrossMinSmem = 120 * 1024;  // keeps the CTA alone on its SM (it holds all of TMEM)
 
+// Separate-P layout (D <= 96, M <= 128): TMEM S0 [0,128), S1 [128,256),
+// O0 [256,256+D), O1 [256+D,256+2D), one 64-column P buffer [256+2D,+64)
+// shared by the two warpgroups (P of tile i is written after P V of tile
+// i-1). S is released as soon as it is loaded, so the next S of a warpgroup
+// is computed while it exponentiates; the output is staged in two buffers of
+// its own, so a query slot returns to the producer as soon as S is done.
+// Otherwise P overwrites S, the warpgroup owns [256g, 256g+256) (S at 0, O at
+// 128) and the output is staged in the slot its queries came from.
+template <int D>
+__host__ __device__ constexpr bool cross_sep_p(int M) {
+  return D <= 96 && M <= 128;
+}
 template <int D>
 __host__ __device__ constexpr int cross_smem_need(int M, int qs) {
-  return 1024 + qs * TileCfg<D>::kTileBytes + 2 * (((M + 31) / 32) * 32) * D * 2 + 256 * 4 + 256;
+  return 1024 + (qs + (cross_sep_p<D>(M) ? 2 : 0)) * TileCfg<D>::kTileBytes + 2 * (((M + 31) / 32) * 32) * D * 2 +
+         128 * 32 + (((M + 31) / 32) * 32) * 32 + 256 * 4 + 256;
 }
 // Slots that fit next to the text keys / values (4 at most, 2 at least).
 template <int D>
@@ -68,7 +87,7 @@ __host__ __device__ constexpr int cross_smem_bytes(int M) {
                                                                   : cross_smem_need<D>(M, cross_slots<D>(M));
 }
 
-template <int D>
+template <int D, bool kSep>
 __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __grid_constant__ CrossParams p) {
   using C = TileCfg<D>;
   constexpr int TB = C::kTileBytes;
@@ -76,22 +95,28 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int QS = p.qs;
   const int Mp = ((p.M + 31) / 32) * 32;
-  uint8_t* sQ = sm;  // QS query-tile slots (also the output staging)
-  uint8_t* sKy = sQ + QS * TB;
+  uint8_t* sQ = sm;  // QS query-tile slots (aliased layout: also the output staging)
+  uint8_t* sOut = sQ + QS * TB;  // separate-P layout: two output staging buffers
+  uint8_t* sKy = sOut + (kSep ? 2 * TB : 0);
   uint8_t* sVy = sKy + Mp * D * 2;
-  float* sw = reinterpret_cast<float*>(sVy + Mp * D * 2);
+  uint8_t* sOnes = sVy + Mp * D * 2;  // 128 rows x 16 bf16 ones (32-byte rows)
+  uint8_t* sBias = sOnes + 128 * 32;  // Mp rows x 16 bf16: 0 (valid key) or -inf
+  float* sw = reinterpret_cast<float*>(sBias + Mp * 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sw + 256);
-  uint64_t* q_full = bars;         // [4]
+  uint64_t* q_full = bars;         // [4] per slot
   uint64_t* q_empty = bars + 4;    // [4]
-  uint64_t* s_full = bars + 8;     // [2] per warpgroup
-  uint64_t* p_full = bars + 10;    // [2]
-  uint64_t* o_full = bars + 12;    // [2]
-  uint64_t* t_free = bars + 14;    // [2] TMEM S / O of the warpgroup read
-  // [4] output tile written to its slot (per slot: a slot's next output
-  // waits for this one's store, so its phases are never skipped)
-  uint64_t* o_staged = bars + 16;
-  uint64_t* drained = bars + 20;  // [2] issuer's MMAs all complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  // [4] output tile written to its staging buffer (per buffer: a buffer's
+  // next output waits for this one's store, so its phases are never skipped)
+  uint64_t* o_staged = bars + 8;
+  uint64_t* s_full = bars + 12;   // [2] per warpgroup
+  uint64_t* s_free = bars + 14;   // [2] S loaded (separate-P layout)
+  uint64_t* p_full = bars + 16;   // [2]
+  uint64_t* pv_done = bars + 18;  // [2] P V complete: the P buffer is free (separate-P layout)
+  uint64_t* o_full = bars + 20;   // [2]
+  uint64_t* t_free = bars + 22;   // [2] the warpgroup's TMEM output (aliased: and S) read
+  uint64_t* drained = bars + 24;  // [2] issuer's MMAs all complete
+  uint64_t* out_free = bars + 26;  // [2] staging buffer read by its store (separate-P layout)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -111,6 +136,11 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
   }
   const int Lp = ((L + 31) / 32) * 32;
 
+  // TMEM columns of warpgroup g's S and O, and of P
+  auto col_S = [](int g) -> uint32_t { return kSep ? 128u * g : 256u * g; };
+  auto col_O = [](int g) -> uint32_t { return kSep ? 256u + static_cast<uint32_t>(D) * g : 256u * g + 128u; };
+  auto col_P = [](int g) -> uint32_t { return kSep ? 256u + 2u * D : 256u * g; };
+
   if (tid == 0) {
     abort_flag = 0;
     for (int i = 0; i < 4; ++i) {
@@ -120,10 +150,13 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&s_full[g], 1);
+      mbar_init(&s_free[g], 128);
       mbar_init(&p_full[g], 128);
+      mbar_init(&pv_done[g], 1);
       mbar_init(&o_full[g], 1);
       mbar_init(&t_free[g], 128);
       mbar_init(&drained[g], 1);
+      mbar_init(&out_free[g], 1);
     }
     fence_mbar_init();
   }
@@ -204,6 +237,14 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
             vv[k];
       }
     }
+    // mask operands (rows are uniform, so the 32-byte swizzle leaves them as
+    // they are)
+    for (int e = ct; e < 128 * 2; e += kCopyThreads)
+      reinterpret_cast<uint4*>(sOnes)[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    for (int e = ct; e < Lp * 2; e += kCopyThreads) {
+      const uint32_t v = (e >> 1) < L ? 0u : 0xFF80FF80u;
+      reinterpret_cast<uint4*>(sBias)[e] = make_uint4(v, v, v, v);
+    }
     for (int j = ct; j < Lp; j += kCopyThreads) {
       float wj = 0.f;
       if (j < L) wj = p.w != nullptr ? __ldg(p.w + static_cast<size_t>(b) * p.M + j) : 1.f / static_cast<float>(L);
@@ -234,38 +275,74 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
     // ------------------------------------------------------------ MMA issuers
     const int g = warp - 1;
     if (lane == 0) {
-      const uint32_t tS = tbase + 256 * g, tO = tS + 128;
+      const uint32_t tS = tbase + col_S(g), tO = tbase + col_O(g), tP = tbase + col_P(g);
       const uint32_t idS = make_idesc_bf16(128, Lp, 0, 0);
       constexpr uint32_t idPV = make_idesc_bf16(128, D, 0, 1);
       const uint32_t aK = smem_u32(sKy), aV = smem_u32(sVy);
-      for (int i = g; i < n_my; i += 2) {
-        const int k = i >> 1, slot = i % QS;
-        if (!mbar_wait(&q_full[slot], (i / QS) & 1, &abort_flag)) break;
-        // the previous tile of this warpgroup has released S (and, when S
-        // reaches into the O columns, its output)
-        if (k > 0) {
-          uint64_t* prev = (has_o && Lp <= 128) ? &o_full[g] : &t_free[g];
-          if (!mbar_wait(prev, (k - 1) & 1, &abort_flag)) break;
-        }
-        tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ + slot * TB);
+      // S_i = Q_i Ky^T (+ the padding mask); the slot returns to the
+      // producer once S_i is done unless the output is staged in it
+      auto issue_S = [&](int i) {
+        const uint32_t aQ = smem_u32(sQ + (i % QS) * TB);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2;
           const uint64_t bd = make_sdesc(aK + c * Mp * 128 + (kk & 3) * 32, 16, 8 * C::row_bytes(c), C::swizzle(c));
           umma_ss(tS, kmajor_desc<D>(aQ, kk), bd, idS, kk > 0 ? 1u : 0u);
         }
+        if (L < Lp)  // padding keys -> -inf
+          umma_ss(tS, make_sdesc(smem_u32(sOnes), 16, 256, kSwizzle32B), make_sdesc(smem_u32(sBias), 16, 256, kSwizzle32B),
+                  idS, 1u);
         umma_commit(&s_full[g]);
-        if (!has_o) {
-          umma_commit(&q_empty[slot]);
-          continue;
-        }
-        if (!mbar_wait(&p_full[g], k & 1, &abort_flag)) break;
-        if (k > 0 && !mbar_wait(&t_free[g], (k - 1) & 1, &abort_flag)) break;
-        tc_fence_after();
+        if (kSep || !has_o) umma_commit(&q_empty[i % QS]);
+      };
+      auto issue_PV = [&]() {
         for (int kk = 0; kk < Lp / 16; ++kk)
-          umma_ts(tO, tS + kk * 8, make_sdesc(aV + kk * 16 * 64, Mp * 64, 512, kSwizzle64B), idPV, kk > 0 ? 1u : 0u);
+          umma_ts(tO, tP + kk * 8, make_sdesc(aV + kk * 16 * 64, Mp * 64, 512, kSwizzle64B), idPV, kk > 0 ? 1u : 0u);
+        if (kSep) umma_commit(&pv_done[g]);
         umma_commit(&o_full[g]);
+      };
+      if constexpr (kSep) {
+        // per tile: the next S as soon as the softmax has loaded the
+        // current one, then P V once P is written
+        bool ok = g < n_my && mbar_wait(&q_full[g % QS], (g / QS) & 1, &abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_S(g);
+        }
+        for (int i = g; ok && i < n_my; i += 2) {
+          const int k = i >> 1;
+          if (i + 2 < n_my) {
+            ok = mbar_wait(&q_full[(i + 2) % QS], ((i + 2) / QS) & 1, &abort_flag) &&
+                 mbar_wait(&s_free[g], k & 1, &abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_S(i + 2);
+          }
+          if (has_o) {
+            ok = mbar_wait(&p_full[g], k & 1, &abort_flag) && (k == 0 || mbar_wait(&t_free[g], (k - 1) & 1, &abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            issue_PV();
+          }
+        }
+      } else {
+        for (int i = g; i < n_my; i += 2) {
+          const int k = i >> 1;
+          if (!mbar_wait(&q_full[i % QS], (i / QS) & 1, &abort_flag)) break;
+          // the previous tile of this warpgroup has released S (and, when S
+          // reaches into the O columns, its output)
+          if (k > 0) {
+            uint64_t* prev = (has_o && Lp <= 128) ? &o_full[g] : &t_free[g];
+            if (!mbar_wait(prev, (k - 1) & 1, &abort_flag)) break;
+          }
+          tc_fence_after();
+          issue_S(i);
+          if (!has_o) continue;
+          if (!mbar_wait(&p_full[g], k & 1, &abort_flag)) break;
+          if (k > 0 && !mbar_wait(&t_free[g], (k - 1) & 1, &abort_flag)) break;
+          tc_fence_after();
+          issue_PV();
+        }
       }
       // every MMA this thread issued has completed before TMEM is released
       umma_commit(&drained[g]);
@@ -275,14 +352,14 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
     // ------------------------------------------------------------ output store
     if (has_o && lane == 0) {
       for (int i = 0; i < n_my; ++i) {
-        const int slot = i % QS;
-        if (!mbar_wait(&o_staged[slot], (i / QS) & 1, &abort_flag)) break;
-        const uint8_t* src = sQ + slot * TB;
+        const int buf = kSep ? (i & 1) : (i % QS);
+        if (!mbar_wait(&o_staged[buf], kSep ? ((i >> 1) & 1) : ((i / QS) & 1), &abort_flag)) break;
+        const uint8_t* src = kSep ? sOut + buf * TB : sQ + buf * TB;
         const int q0 = (tile0 + i) * 128;
         for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&p.o_map[c], src + C::chunk_off(c), 64 * c, h, q0, b);
         bulk_commit_group();
         bulk_wait_read_all();
-        mbar_arrive(&q_empty[slot]);
+        mbar_arrive(kSep ? &out_free[buf] : &q_empty[buf]);
       }
       bulk_wait_all();
     }
@@ -294,65 +371,62 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tbase + 256 * g + lane_addr;
-    const uint32_t tO = tS + 128;
+    const uint32_t tS = tbase + col_S(g) + lane_addr;
+    const uint32_t tO = tbase + col_O(g) + lane_addr;
+    const uint32_t tP = tbase + col_P(g) + lane_addr;
     const float sl2 = p.scale_log2;
-    for (int i = g; i < n_my; i += 2) {
+    float linv_even = 1.f, linv_odd = 1.f;  // 1 / l of this warpgroup's last two tiles
+
+    // softmax of tile i: probabilities, l and the PCSP partial; P -> TMEM
+    auto softmax = [&](int i) -> bool {
       const int k = i >> 1;
       const int q_row = (tile0 + i) * 128 + row;
-      const bool valid = q_row < p.nq;
-      if (!warp_wait(&s_full[g], k & 1, &abort_flag)) break;
+      if (!warp_wait(&s_full[g], k & 1, &abort_flag)) return false;
       tc_fence_after();
       float l = 0.f, score = 0.f;
-      if (Lp <= 128) {
-        // all of S in registers: one TMEM pass. Only the last 32-key chunk
-        // can hold padding keys; they are set to -inf (their weights are 0).
-        uint32_t sr[128];
-        const int nc = Lp / 32;
+      // all of S in registers: one TMEM pass (padding keys hold -inf and
+      // weight 0), specialised on the number NC of 32-key chunks so that
+      // every register index is static
+      auto one_pass = [&](auto nc_tag) -> bool {
+        constexpr int NC = decltype(nc_tag)::value;
+        uint32_t sr[32 * NC];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < nc) tmem_ld32(tS + 32 * c, sr + 32 * c);
+        for (int c = 0; c < NC; ++c) tmem_ld32(tS + 32 * c, sr + 32 * c);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < nc) tmem_ld_wait32(sr + 32 * c);  // ties the loaded registers to the wait
-        if (!has_o) {
+        for (int c = 0; c < NC; ++c) tmem_ld_wait32(sr + 32 * c);  // ties the loaded registers to the wait
+        if (kSep || !has_o) {
           tc_fence_before();
-          mbar_arrive(&t_free[g]);
+          mbar_arrive(kSep ? &s_free[g] : &t_free[g]);  // S may be overwritten
         }
-#pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (j >= L) sr[j] = __float_as_uint(-INFINITY);
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < nc) {
+        for (int j = 0; j < 32 * NC; j += 8)
 #pragma unroll
-            for (int i2 = 0; i2 < 32; i2 += 8)
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                m4[q] = fmax3(m4[q], __uint_as_float(sr[32 * c + i2 + 2 * q]), __uint_as_float(sr[32 * c + i2 + 2 * q + 1]));
-          }
-        }
+          for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(sr[j + 2 * q]), __uint_as_float(sr[j + 2 * q + 1]));
         const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         const uint64_t sl2x2 = f2_pack(sl2, sl2), neg2 = f2_pack(-mx * sl2, -mx * sl2);
         uint64_t lacc[2] = {0, 0}, sacc[2] = {0, 0};  // packed row sums and weighted sums
+        uint32_t pk[16 * NC];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c >= nc) continue;
-          uint32_t pk[16];
+        for (int i2 = 0; i2 < 16 * NC; ++i2) {
+          const int j0 = 2 * i2;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), sl2x2, neg2), x0, x1);
+          const float a = ex2_approx(x0), bb = ex2_approx(x1);
+          const uint64_t e2 = f2_pack(a, bb);
+          const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
+          lacc[i2 & 1] = f2_add(lacc[i2 & 1], e2);
+          sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+          pk[i2] = pack_bf16x2(a, bb);
+          if (!kSep && has_o && (i2 & 15) == 15) tmem_st16(tP + (i2 - 15), pk + (i2 - 15));
+        }
+        if (kSep && has_o) {
+          // the shared P buffer: tile i-1's P V (the other warpgroup) has
+          // read it
+          if (i > 0 && !warp_wait(&pv_done[g ^ 1], ((i - 1) >> 1) & 1, &abort_flag)) return false;
+          tc_fence_after();
 #pragma unroll
-          for (int i2 = 0; i2 < 16; ++i2) {
-            const int j0 = 32 * c + 2 * i2;
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), sl2x2, neg2), x0, x1);
-            const float a = ex2_approx(x0), bb = ex2_approx(x1);
-            const uint64_t e2 = f2_pack(a, bb);
-            const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
-            lacc[i2 & 1] = f2_add(lacc[i2 & 1], e2);
-            sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
-            pk[i2] = pack_bf16x2(a, bb);
-          }
-          if (has_o) tmem_st16(tS + 16 * c, pk);
+          for (int c = 0; c < NC; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
         }
         float l0, l1, l2, l3, s0, s1, s2, s3;
         f2_unpack(lacc[0], l0, l1);
@@ -361,8 +435,21 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         f2_unpack(sacc[1], s2, s3);
         l = (l0 + l1) + (l2 + l3);
         score = (s0 + s1) + (s2 + s3);
+        return true;
+      };
+      if (Lp <= 128) {
+        bool ok;
+        switch (Lp / 32) {
+          case 1: ok = one_pass(std::integral_constant<int, 1>{}); break;
+          case 2: ok = one_pass(std::integral_constant<int, 2>{}); break;
+          case 3: ok = one_pass(std::integral_constant<int, 3>{}); break;
+          default: ok = one_pass(std::integral_constant<int, 4>{}); break;
+        }
+        if (!ok) return false;
       } else {
-        // pass 1: row max over valid keys
+        // (aliased layout only) pass 1: row max over valid keys (the key
+        // tests are redundant with the -inf columns but keep this path's
+        // registers low)
         float mx = -INFINITY;
         for (int c = 0; c < Lp / 32; ++c) {
           uint32_t sr[32];
@@ -390,7 +477,7 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
             score = fmaf(sw[j0 + 1], bb, score);
             pk[i2] = pack_bf16x2(a, bb);
           }
-          if (has_o) tmem_st16(tS + 16 * c, pk);
+          if (has_o) tmem_st16(tP + 16 * c, pk);
         }
         if (!has_o) {
           tc_fence_before();
@@ -402,15 +489,22 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         tc_fence_before();
         mbar_arrive(&p_full[g]);
       }
-      if (p.partial != nullptr && valid) p.partial[(static_cast<size_t>(b) * p.H + h) * p.nq + q_row] = score / l;
-      if (!has_o) continue;
+      if (p.partial != nullptr && q_row < p.nq) p.partial[(static_cast<size_t>(b) * p.H + h) * p.nq + q_row] = score / l;
+      if (k & 1) linv_odd = 1.f / l;
+      else linv_even = 1.f / l;
+      return true;
+    };
 
-      // O = P Vy / l -> bf16 into the slot of this tile's queries (the S
-      // product has read them), laid out like a query tile for the store
-      if (!warp_wait(&o_full[g], k & 1, &abort_flag)) break;
+    // O = P Vy / l of tile i -> bf16 into a staging buffer laid out like a
+    // query tile for the store: the warpgroup's own (separate-P layout) or
+    // the slot of the tile's queries, which the S product has read
+    auto epilogue = [&](int i) -> bool {
+      const int k = i >> 1;
+      if (!warp_wait(&o_full[g], k & 1, &abort_flag)) return false;
+      if (kSep && k > 0 && !warp_wait(&out_free[g], (k - 1) & 1, &abort_flag)) return false;
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      uint8_t* slot = sQ + (i % QS) * TB;
+      const float inv_l = (k & 1) ? linv_odd : linv_even;
+      uint8_t* slot = kSep ? sOut + g * TB : sQ + (i % QS) * TB;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -435,7 +529,23 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&o_staged[i % QS]);
+      mbar_arrive(&o_staged[kSep ? g : i % QS]);
+      return true;
+    };
+
+    if constexpr (kSep) {
+      // softmax of the next tile before the output of the previous one: its
+      // P V has long finished by then
+      for (int i = g;; i += 2) {
+        if (i < n_my && !softmax(i)) break;
+        if (has_o && i >= 2 && i - 2 < n_my && !epilogue(i - 2)) break;
+        if (i >= n_my) break;
+      }
+    } else {
+      for (int i = g; i < n_my; i += 2) {
+        if (!softmax(i)) break;
+        if (has_o && !epilogue(i)) break;
+      }
     }
   }
 

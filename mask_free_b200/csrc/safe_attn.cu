@@ -208,7 +208,12 @@ safe_status launch_cross(CrossParams& p, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(cross_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kCrossMaxSmem);
+    attr_err = cudaFuncSetAttribute(cross_attn_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kCrossMaxSmem);
+    if constexpr (D <= 96)
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(cross_attn_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kCrossMaxSmem);
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   // one CTA per SM (each holds all of TMEM), a few per (b, h), each streaming
@@ -218,7 +223,14 @@ safe_status launch_cross(CrossParams& p, cudaStream_t s) {
   per_bh = per_bh < 1 ? 1 : (per_bh > n_tiles ? n_tiles : per_bh);
   p.qs = cross_slots<D>(p.M);
   dim3 grid(per_bh, p.H, p.B);
-  cross_attn_kernel<D><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
+  bool launched = false;
+  if constexpr (D <= 96) {
+    if (cross_sep_p<D>(p.M)) {
+      cross_attn_kernel<D, true><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
+      launched = true;
+    }
+  }
+  if (!launched) cross_attn_kernel<D, false><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
   return launch_status();
 }
 
