@@ -561,8 +561,17 @@ __global__ void pcsp_reduce_kernel(const float* __restrict__ partial, float* __r
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const int b = blockIdx.y;
   if (i >= N) return;
+  // eight heads' loads in flight at a time, summed in head order
+  const float* src = partial + static_cast<size_t>(b) * H * N + i;
   float acc = 0.f;
-  for (int h = 0; h < H; ++h) acc += partial[(static_cast<size_t>(b) * H + h) * N + i];
+  for (int h0 = 0; h0 < H; h0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = h0 + u < H ? __ldg(src + static_cast<size_t>(h0 + u) * N) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (h0 + u < H) acc += v[u];
+  }
   acc = acc / static_cast<float>(H);
   float* dst = scores + static_cast<size_t>(b) * N + i;
   *dst = accumulate ? *dst + acc : acc;
