@@ -315,3 +315,101 @@ def cache_scatter(cache: np.ndarray, src: np.ndarray, S: Optional[np.ndarray],
         for r in range(S.shape[1]):
             out[b, S[b, r]] = src[b, r] if src_compact else src[b, S[b, r]]
     return out
+
+
+# ----------------------------------------------------------------------------
+# Sensitivity field on the latent grid  (Eq. (11))
+# ----------------------------------------------------------------------------
+
+
+def gaussian_taps(sigma: float, truncate: float = 4.0) -> np.ndarray:
+    """The 1-D Gaussian G_sigma of Eq. (11) at integer offsets t = -r..r.
+
+    Weights exp(-t^2 / (2 sigma^2)) normalised to sum 1, cut at radius
+    r = floor(truncate * sigma + 1/2). The paper gives no sigma and no
+    cut-off; a cut at 4 sigma is the usual choice. sigma = 0 is the identity.
+    """
+    if sigma <= 0.0:
+        return np.ones(1, dtype=np.float64)
+    r = int(math.floor(truncate * sigma + 0.5))
+    t = np.arange(-r, r + 1, dtype=np.float64)
+    g = np.exp(-(t * t) / (2.0 * sigma * sigma))
+    return g / np.sum(g)
+
+
+def reflect_index(idx: np.ndarray, n: int) -> np.ndarray:
+    """Index into [0, n) of the half-sample symmetric extension of a line of
+    n values: ... x1 x0 | x0 x1 ... x_{n-1} | x_{n-1} x_{n-2} ... (period 2n)."""
+    m = np.mod(np.asarray(idx), 2 * n)
+    return np.where(m < n, m, 2 * n - 1 - m)
+
+
+def smooth_scores(scores: np.ndarray, grid_h: int, grid_w: int, sigma: float,
+                  truncate: float = 4.0) -> np.ndarray:
+    """G_sigma * s~ of Eq. (11), per sample.
+
+    The N = grid_h * grid_w scores of a sample lie on the latent token grid
+    in row-major order (token i = y * grid_w + x). The 2-D Gaussian is
+    separable: convolve every row with the 1-D taps, then every column.
+    Borders: half-sample reflection (the paper names no border rule).
+    """
+    s = np.asarray(scores, dtype=np.float64)
+    B, N = s.shape
+    assert N == grid_h * grid_w
+    g = gaussian_taps(sigma, truncate)
+    r = (g.size - 1) // 2
+    f = s.reshape(B, grid_h, grid_w)
+    xs, ys = np.arange(grid_w), np.arange(grid_h)
+    rows = np.zeros_like(f)
+    for t in range(-r, r + 1):
+        rows += g[t + r] * f[:, :, reflect_index(xs + t, grid_w)]
+    out = np.zeros_like(f)
+    for t in range(-r, r + 1):
+        out += g[t + r] * rows[:, reflect_index(ys + t, grid_h), :]
+    return out.reshape(B, N)
+
+
+def norm01(x: np.ndarray) -> np.ndarray:
+    """Norm of Eq. (11): per-sample min-max map onto [0, 1]. A flat field
+    (max = min) maps to 0, a reading: the paper does not define that case."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    for b in range(x.shape[0]):
+        lo, hi = np.min(x[b]), np.max(x[b])
+        if hi > lo:
+            out[b] = (x[b] - lo) / (hi - lo)
+    return out
+
+
+def sensitivity_field(scores: np.ndarray, grid_h: int, grid_w: int, sigma: float,
+                      truncate: float = 4.0) -> np.ndarray:
+    """s = Norm(G_sigma * s~), Eq. (11). [B, N] -> [B, N] in [0, 1]."""
+    return norm01(smooth_scores(scores, grid_h, grid_w, sigma, truncate))
+
+
+# ----------------------------------------------------------------------------
+# Sensitivity-weighted CFG  (Eq. (20), (21))
+# ----------------------------------------------------------------------------
+
+
+def partition_indicator(S: np.ndarray, N: int) -> np.ndarray:
+    """The binary variant after Eq. (21): s_i = 1 for tokens of S, 0 for C."""
+    S = np.asarray(S)
+    out = np.zeros((S.shape[0], N), dtype=np.float64)
+    for b in range(S.shape[0]):
+        out[b, S[b]] = 1.0
+    return out
+
+
+def sw_cfg(f_c: np.ndarray, f_u: np.ndarray, s: np.ndarray, gamma_ctx: float,
+           gamma_sens: float) -> np.ndarray:
+    """Eq. (20): gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) * s_i, then
+    Eq. (21): f^_i = f_u,i + gamma_i * (f_c,i - f_u,i).
+
+    f_c, f_u: conditional / unconditional predictions [B, N, C] (token-major,
+    C values per token); s: [B, N]. Returns [B, N, C] in fp64.
+    """
+    fc = np.asarray(f_c, dtype=np.float64)
+    fu = np.asarray(f_u, dtype=np.float64)
+    gamma = gamma_ctx + (gamma_sens - gamma_ctx) * np.asarray(s, dtype=np.float64)
+    return fu + gamma[:, :, None] * (fc - fu)

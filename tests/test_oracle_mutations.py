@@ -72,8 +72,50 @@ def _scatter_off_by_one(cache, src, Sidx, src_compact):
     return out
 
 
+def _reflect_whole_sample(idx, n):
+    # mirror about the edge sample itself (x1 x0 | x0 is not repeated): a
+    # different border rule
+    if n == 1:
+        return np.zeros_like(np.asarray(idx))
+    m = np.mod(np.asarray(idx), 2 * n - 2)
+    return np.where(m < n, m, 2 * n - 2 - m)
+
+
+def _taps_unnormalised(sigma, truncate=4.0):
+    g = _ORIG["gaussian_taps"](sigma, truncate)
+    return g / g.max()
+
+
+def _smooth_swapped_axes(scores, grid_h, grid_w, sigma, truncate=4.0):
+    # grid height and width exchanged (rows of the wrong length)
+    return _ORIG["smooth_scores"](scores, grid_w, grid_h, sigma, truncate)
+
+
+def _norm_no_min(x):
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    for b in range(x.shape[0]):
+        hi = np.max(x[b])
+        if hi != 0:
+            out[b] = x[b] / hi
+    return out
+
+
+def _sw_cfg_swapped(f_c, f_u, s, gamma_ctx, gamma_sens):
+    return _ORIG["sw_cfg"](f_u, f_c, s, gamma_ctx, gamma_sens)
+
+
+def _sw_cfg_scales_swapped(f_c, f_u, s, gamma_ctx, gamma_sens):
+    return _ORIG["sw_cfg"](f_c, f_u, s, gamma_sens, gamma_ctx)
+
+
+def _indicator_complement(S, N):
+    return 1.0 - _ORIG["partition_indicator"](S, N)
+
+
 _ORIG = {n: getattr(S, n) for n in ("attention", "softmax_rows", "ceil_k", "topk_partition", "row_in_R",
-                                    "pcsp_scores", "cache_scatter")}
+                                    "pcsp_scores", "cache_scatter", "gaussian_taps", "smooth_scores", "sw_cfg",
+                                    "partition_indicator")}
 
 MUTATIONS = {
     "attention_no_scale": ("attention", _attention_no_scale),
@@ -85,6 +127,13 @@ MUTATIONS = {
     "classifier_ignores_nonfinite": ("row_in_R", _row_in_R_no_finite),
     "pcsp_missing_head_mean": ("pcsp_scores", _pcsp_no_mean),
     "scatter_off_by_one": ("cache_scatter", _scatter_off_by_one),
+    "smoothing_whole_sample_reflection": ("reflect_index", _reflect_whole_sample),
+    "smoothing_unnormalised_taps": ("gaussian_taps", _taps_unnormalised),
+    "smoothing_swapped_grid_axes": ("smooth_scores", _smooth_swapped_axes),
+    "norm_without_min": ("norm01", _norm_no_min),
+    "sw_cfg_swapped_predictions": ("sw_cfg", _sw_cfg_swapped),
+    "sw_cfg_swapped_scales": ("sw_cfg", _sw_cfg_scales_swapped),
+    "indicator_complement": ("partition_indicator", _indicator_complement),
 }
 
 
@@ -102,6 +151,10 @@ def _run_all_pins():
         elif fn.__name__ == "test_ceil_k_golden":
             params = json.load(open(os.path.join(golden, "topk_k_values.json")))["cases"]
         calls = [(c,) for c in params] if params else [()]
+        for mark in getattr(fn, "pytestmark", []):
+            if mark.name == "parametrize" and not params:
+                multi = "," in mark.args[0]
+                calls = [tuple(v) if multi else (v,) for v in mark.args[1]]
         for args in calls:
             try:
                 fn(*args)

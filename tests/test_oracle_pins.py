@@ -413,3 +413,97 @@ def test_topk_all_equal_and_signed_zero():
     assert list(S[0]) == [0, 1, 4]
     S, C = O.topk_partition(np.arange(6, dtype=float).reshape(1, 6), 6)
     assert list(S[0]) == list(range(6)) and C.shape == (1, 0)
+
+
+# ---------------------------------------------------------------- Eq. (11): smoothing and Norm
+
+
+@pytest.mark.parametrize("shape,sigma", [((16, 16), 0.5), ((12, 20), 1.0), ((20, 12), 2.5), ((9, 7), 7.0)])
+def test_smoothing_matches_library_gaussian_filter(shape, sigma):
+    # an independent implementation of the same operator: scipy's separable
+    # Gaussian filter, half-sample reflection at the borders, cut at 4 sigma
+    # (non-square grids catch a swapped axis; sigma = 7 on a 9 x 7 grid needs
+    # repeated reflections)
+    from scipy.ndimage import gaussian_filter
+    gh, gw = shape
+    rng = np.random.default_rng(11)
+    s = rng.random((2, gh * gw))
+    got = O.smooth_scores(s, gh, gw, sigma)
+    for b in range(2):
+        ref = gaussian_filter(s[b].reshape(gh, gw), sigma, mode="reflect", truncate=4.0)
+        np.testing.assert_allclose(got[b].reshape(gh, gw), ref, rtol=0, atol=1e-13)
+
+
+def test_smoothing_identity_constant_and_interior_impulse():
+    rng = np.random.default_rng(12)
+    s = rng.random((1, 35))
+    np.testing.assert_array_equal(O.smooth_scores(s, 5, 7, 0.0), s)  # sigma = 0: no smoothing
+    c = np.full((1, 48), 0.37)
+    np.testing.assert_allclose(O.smooth_scores(c, 6, 8, 1.3), c, atol=1e-15)  # a flat field stays flat
+    # an impulse far from the borders spreads into the sampled 2-D Gaussian:
+    # value at offset (dy, dx) = exp(-(dy^2 + dx^2) / (2 sigma^2)) / Z^2, total 1
+    gh = gw = 33
+    sigma = 1.5
+    d = np.zeros((1, gh * gw))
+    d[0, 16 * gw + 16] = 1.0
+    out = O.smooth_scores(d, gh, gw, sigma).reshape(gh, gw)
+    z = sum(math.exp(-t * t / (2 * sigma * sigma)) for t in range(-6, 7))  # radius floor(4 * 1.5 + 0.5) = 6
+    for dy, dx in [(0, 0), (1, 0), (0, 2), (3, -4), (-6, 6)]:
+        want = math.exp(-(dy * dy + dx * dx) / (2 * sigma * sigma)) / (z * z)
+        assert abs(out[16 + dy, 16 + dx] - want) < 1e-15
+    assert out[16 + 7, 16] == 0.0 and abs(out.sum() - 1.0) < 1e-13
+
+
+def test_norm_maps_onto_unit_interval_preserving_order():
+    rng = np.random.default_rng(13)
+    x = rng.normal(size=(3, 50)) * 7 + 2
+    y = O.norm01(x)
+    for b in range(3):
+        assert y[b].min() == 0.0 and y[b].max() == 1.0
+        assert np.array_equal(np.argsort(x[b], kind="stable"), np.argsort(y[b], kind="stable"))
+        i, j = np.argmin(x[b]), np.argmax(x[b])
+        k = (i + 1) % 50 if (i + 1) % 50 != j else (i + 2) % 50
+        # affine: the relative position of any value between min and max
+        assert abs(y[b, k] - (x[b, k] - x[b, i]) / (x[b, j] - x[b, i])) < 1e-15
+    assert np.array_equal(O.norm01(np.full((1, 4), 5.0)), np.zeros((1, 4)))
+    # top-k is unchanged by Norm (a strictly increasing map)
+    S1, _ = O.topk_partition(x, 9)
+    S2, _ = O.topk_partition(y, 9)
+    assert np.array_equal(S1, S2)
+
+
+# ---------------------------------------------------------------- Eq. (20), (21): SW-CFG
+
+
+def test_sw_cfg_special_cases_and_interpolation():
+    rng = np.random.default_rng(14)
+    fc, fu = rng.normal(size=(2, 6, 3)), rng.normal(size=(2, 6, 3))
+    s = rng.random((2, 6))
+    # gamma = 1 everywhere returns the conditional prediction, 0 the
+    # unconditional one (whatever s is)
+    np.testing.assert_allclose(O.sw_cfg(fc, fu, s, 1.0, 1.0), fc, atol=1e-15)
+    np.testing.assert_allclose(O.sw_cfg(fc, fu, s, 0.0, 0.0), fu, atol=1e-15)
+    # s = 0 uses the context scale, s = 1 the sensitive scale: with the other
+    # scale arbitrary, the conditional / unconditional prediction comes back
+    np.testing.assert_allclose(O.sw_cfg(fc, fu, np.zeros((2, 6)), 1.0, 9.0), fc, atol=1e-15)
+    np.testing.assert_allclose(O.sw_cfg(fc, fu, np.ones((2, 6)), -3.0, 0.0), fu, atol=1e-15)
+    # the guided prediction is the extrapolation (1 - g) f_u + g f_c, affine in s
+    g_ctx, g_sens = 4.0, 7.5
+    out = O.sw_cfg(fc, fu, s, g_ctx, g_sens)
+    g = g_ctx * (1 - s) + g_sens * s
+    np.testing.assert_allclose(out, (1 - g)[..., None] * fu + g[..., None] * fc, atol=1e-12)
+    mid = O.sw_cfg(fc, fu, np.full((2, 6), 0.5), g_ctx, g_sens)
+    ends = 0.5 * (O.sw_cfg(fc, fu, np.zeros((2, 6)), g_ctx, g_sens) + O.sw_cfg(fc, fu, np.ones((2, 6)), g_ctx, g_sens))
+    np.testing.assert_allclose(mid, ends, atol=1e-12)
+
+
+def test_partition_indicator_binary_variant():
+    S = np.array([[0, 3, 4], [1, 2, 5]])
+    ind = O.partition_indicator(S, 6)
+    assert ind.tolist() == [[1, 0, 0, 1, 1, 0], [0, 1, 1, 0, 0, 1]]
+    rng = np.random.default_rng(15)
+    fc, fu = rng.normal(size=(2, 6, 2)), rng.normal(size=(2, 6, 2))
+    out = O.sw_cfg(fc, fu, ind, 1.0, 0.0)  # C tokens keep f_c, S tokens get f_u
+    for b in range(2):
+        for i in range(6):
+            np.testing.assert_allclose(out[b, i], fu[b, i] if i in S[b] else fc[b, i], atol=1e-15)
