@@ -297,6 +297,23 @@ def kernel_table(dev, pk):
             Ck = torch.empty((s.B, s.N - k), dtype=torch.int32, device=dev)
             t_t = time_kernel(lambda: ops.topk_partition(sc, k, S=Sk, C=Ck))
             out["topk"] = {"ms": t_t}
+            # sensitivity field (Eq. (11)) of the PCSP scores on the 160 x 160
+            # latent grid, and SW-CFG (Eq. (20), (21)) of one CFG pair with 16
+            # prediction values per token (2 x 2 patch x 4 latent channels)
+            side = int(math.isqrt(s.N))
+            if side * side == s.N:
+                sf = torch.empty_like(sc)
+                wsf = torch.empty(ops.sensitivity_workspace_bytes(s.B, s.N), dtype=torch.uint8, device=dev)
+                t_f = time_kernel(lambda: ops.sensitivity_field(sc, side, side, 2.0, out=sf, ws=wsf))
+                out["sensitivity_field"] = {"ms": t_f, "grid": f"{side}x{side}", "sigma": 2.0,
+                                            "gbs": 5 * 4 * s.B * s.N / t_f / 1e6}
+                for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+                    fc = torch.randn((1, s.N, 16), device=dev).to(dt)
+                    fu = torch.randn((1, s.N, 16), device=dev).to(dt)
+                    fo = torch.empty_like(fc)
+                    t_g = time_kernel(lambda: ops.sw_cfg(fc, fu, sf[:1], 4.0, 7.5, out=fo))
+                    gb = 3 * fc.numel() * fc.element_size() + 4 * s.N
+                    out[f"sw_cfg_{tag}"] = {"ms": t_g, "gbs": gb / t_g / 1e6, "pct_hbm": 100 * gb / t_g / 1e6 / pk["hbm"]}
             # SRSU wall time against |S|/N
             sweep = {}
             for rho in (0.1, 0.2, 0.3, 0.5, 1.0):

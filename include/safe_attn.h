@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { SAFE_BOOL = 0, SAFE_U8 = 1, SAFE_F32 = 2, SAFE_F16 = 3, SAFE_BF16 = 4 } safe_dtype;
 
-/* ABI version of this header (bumped on any signature change): 2. */
+/* ABI version of this header (bumped on any signature or entry-point change): 3. */
 int safe_abi_version(void);
 const char* safe_status_string(int status);
 
@@ -217,6 +217,51 @@ safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k
  */
 safe_status safe_ctx_cache_scatter(const void* Ksrc, const void* Vsrc, int src_compact, const int32_t* S, int k,
                                    void* Kc, void* Vc, int B, int N, int H, int d, void* stream);
+
+/*
+ * Sensitivity field of Eq. (11):  s = Norm(G_sigma * s~)  per sample.
+ * The N = grid_h * grid_w scores of a sample (e.g. from safe_pcsp_topk) lie
+ * on the latent token grid in row-major order (token i = y * grid_w + x).
+ * G_sigma: the separable Gaussian exp(-t^2 / (2 sigma^2)) at integer offsets
+ * |t| <= r = floor(truncate * sigma + 1/2), normalised to sum 1 (sigma = 0:
+ * no smoothing); borders by half-sample reflection. Norm: per-sample min-max
+ * map onto [0, 1]; a flat field maps to 0. The paper gives neither sigma nor
+ * the border rule; both are inputs / stated readings. fp32 arithmetic.
+ *  scores  device fp32 [B, N] (read); s device fp32 [B, N] (written; may
+ *          not alias scores).
+ *  ws      device workspace of safe_sensitivity_workspace_bytes(B, N) bytes
+ *          (256-byte aligned); contents need no initialisation.
+ *  sigma >= 0 and truncate > 0, finite, with r <= 128 (else
+ *  SAFE_ERR_UNSUPPORTED). Top-k of s (Eq. (12)) with safe_topk_partition.
+ */
+size_t safe_sensitivity_workspace_bytes(int B, int N);
+safe_status safe_sensitivity_field(const float* scores, float* s, int B, int grid_h, int grid_w, float sigma,
+                                   float truncate, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Binary sensitivity field of the SW-CFG binary variant (after Eq. (21)):
+ * s[b, i] = 1 for i in S[b], 0 for the context tokens C.
+ *  S  device int32 [B, k], strictly ascending, values in [0, N) (violations
+ *     are flagged, SAFE_ERR_DEVICE_CHECK); s device fp32 [B, N] (written).
+ */
+safe_status safe_partition_indicator(const int32_t* S, int k, float* s, int B, int N, void* stream);
+
+/*
+ * Sensitivity-weighted classifier-free guidance, Eq. (20), (21):
+ *   gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) * s[b, i]
+ *   out[b, i, c] = f_u[b, i, c] + gamma_i * (f_c[b, i, c] - f_u[b, i, c])
+ * gamma_sens == gamma_ctx is standard CFG with that scale.
+ *  f_c, f_u  device [B, N, C] conditional / unconditional predictions
+ *            (token-major, C values per token), dtype SAFE_F32 or SAFE_BF16
+ *            (naturally aligned; 16-byte vectors are used when every row
+ *            and pointer allows).
+ *  s         device fp32 [B, N] (e.g. from safe_sensitivity_field or
+ *            safe_partition_indicator).
+ *  out       device [B, N, C], same dtype; may alias f_c or f_u.
+ * fp32 arithmetic; bf16 output rounded to nearest even.
+ */
+safe_status safe_sw_cfg(const void* f_c, const void* f_u, const float* s, void* out, int dtype, int B, int N, int C,
+                        float gamma_ctx, float gamma_sens, void* stream);
 
 /*
  * Device status word: synchronises `stream`, writes to *h_status (host) the

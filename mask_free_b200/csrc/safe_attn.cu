@@ -16,12 +16,13 @@
 #include "flash_attn.cuh"
 #include "cross_attn.cuh"
 #include "aux_kernels.cuh"
+#include "guidance.cuh"
 
 using namespace safe;
 
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -519,6 +520,93 @@ safe_status safe_ctx_cache_scatter(const void* Ksrc, const void* Vsrc, int src_c
   cache_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
       static_cast<const uint4*>(Ksrc), static_cast<const uint4*>(Vsrc), src_compact, S, k, static_cast<uint4*>(Kc),
       static_cast<uint4*>(Vc), B, N, row_units);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- sensitivity field and SW-CFG
+size_t safe_sensitivity_workspace_bytes(int B, int N) {
+  if (B < 1 || N < 1) return 0;
+  return align256(static_cast<size_t>(B) * N * sizeof(float)) + align256(static_cast<size_t>(B) * 2 * sizeof(uint32_t));
+}
+
+safe_status safe_sensitivity_field(const float* scores, float* s, int B, int grid_h, int grid_w, float sigma,
+                                   float truncate, void* ws, size_t ws_bytes, void* stream) {
+  if (scores == nullptr || s == nullptr || scores == s || B < 1 || B > 65535 || grid_h < 1 || grid_w < 1)
+    return SAFE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(grid_h) * grid_w > INT_MAX / 2) return SAFE_ERR_INVALID_ARG;
+  if (!std::isfinite(sigma) || sigma < 0.f || !std::isfinite(truncate) || truncate <= 0.f) return SAFE_ERR_INVALID_ARG;
+  const int N = grid_h * grid_w;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < safe_sensitivity_workspace_bytes(B, N))
+    return SAFE_ERR_INVALID_ARG;
+  SmoothParams p{};
+  // the taps of G_sigma, in double, then rounded to fp32
+  const double r_real = sigma > 0.f ? std::floor(static_cast<double>(truncate) * sigma + 0.5) : 0.0;
+  if (r_real > kMaxSmoothRadius) return SAFE_ERR_UNSUPPORTED;
+  p.r = static_cast<int>(r_real);
+  if (p.r == 0) {
+    p.taps[0] = 1.f;
+  } else {
+    double g[kMaxTaps], sum = 0.0;
+    for (int t = -p.r; t <= p.r; ++t) {
+      g[t + p.r] = std::exp(-(static_cast<double>(t) * t) / (2.0 * sigma * sigma));
+      sum += g[t + p.r];
+    }
+    for (int t = 0; t <= 2 * p.r; ++t) p.taps[t] = static_cast<float>(g[t] / sum);
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.in = scores;
+  p.rows = reinterpret_cast<float*>(w);
+  p.out = s;
+  p.minmax = reinterpret_cast<uint32_t*>(w + align256(static_cast<size_t>(B) * N * sizeof(float)));
+  p.B = B;
+  p.gh = grid_h;
+  p.gw = grid_w;
+  cudaStream_t st = as_stream(stream);
+  const dim3 grid((N + 255) / 256, B);
+  smooth_rows_kernel<<<grid, 256, 0, st>>>(p);
+  smooth_cols_kernel<<<grid, 256, 0, st>>>(p);
+  norm01_kernel<<<grid, 256, 0, st>>>(s, p.minmax, N);
+  return launch_status();
+}
+
+safe_status safe_partition_indicator(const int32_t* S, int k, float* s, int B, int N, void* stream) {
+  if (S == nullptr || s == nullptr || B < 1 || B > 65535 || N < 1 || k < 1 || k > N) return SAFE_ERR_INVALID_ARG;
+  partition_indicator_kernel<<<dim3((N + 255) / 256, B), 256, 0, as_stream(stream)>>>(S, k, s, N);
+  return launch_status();
+}
+
+safe_status safe_sw_cfg(const void* f_c, const void* f_u, const float* s, void* out, int dtype, int B, int N, int C,
+                        float gamma_ctx, float gamma_sens, void* stream) {
+  if (f_c == nullptr || f_u == nullptr || s == nullptr || out == nullptr || B < 1 || N < 1 || C < 1)
+    return SAFE_ERR_INVALID_ARG;
+  if (dtype != SAFE_F32 && dtype != SAFE_BF16) return SAFE_ERR_UNSUPPORTED;
+  if (!std::isfinite(gamma_ctx) || !std::isfinite(gamma_sens)) return SAFE_ERR_INVALID_ARG;
+  const size_t esize = dtype == SAFE_F32 ? 4 : 2;
+  auto aligned = [](const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+  if (!aligned(f_c, esize) || !aligned(f_u, esize) || !aligned(out, esize) || !aligned(s, 4))
+    return SAFE_ERR_INVALID_ARG;
+  const size_t total = static_cast<size_t>(B) * N * C;
+  const int vec = static_cast<int>(16 / esize);
+  const bool vec_ok = (C % vec) == 0 && aligned(f_c, 16) && aligned(f_u, 16) && aligned(out, 16);
+  const size_t n_vec = vec_ok ? total / vec : total;
+  const size_t want = (n_vec + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(want < static_cast<size_t>(device_sms()) * 16 ? (want ? want : 1)
+                                                                                          : static_cast<size_t>(device_sms()) * 16);
+  const float diff = gamma_sens - gamma_ctx;
+  cudaStream_t st = as_stream(stream);
+  if (dtype == SAFE_F32) {
+    auto fc = static_cast<const float*>(f_c);
+    auto fu = static_cast<const float*>(f_u);
+    auto o = static_cast<float*>(out);
+    if (vec_ok) sw_cfg_kernel<float, 4><<<blocks, 256, 0, st>>>(fc, fu, s, o, n_vec, C, gamma_ctx, diff);
+    else sw_cfg_kernel<float, 1><<<blocks, 256, 0, st>>>(fc, fu, s, o, n_vec, C, gamma_ctx, diff);
+  } else {
+    auto fc = static_cast<const __nv_bfloat16*>(f_c);
+    auto fu = static_cast<const __nv_bfloat16*>(f_u);
+    auto o = static_cast<__nv_bfloat16*>(out);
+    if (vec_ok) sw_cfg_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(fc, fu, s, o, n_vec, C, gamma_ctx, diff);
+    else sw_cfg_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>(fc, fu, s, o, n_vec, C, gamma_ctx, diff);
+  }
   return launch_status();
 }
 

@@ -41,8 +41,12 @@ _SIGS = {
     "safe_status_string": [_i],
     "safe_selftest_wait_timeout": [ctypes.c_uint64, _vp],
     "safe_pcsp_topk_noalloc": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
+    "safe_sensitivity_workspace_bytes": [_i, _i],
+    "safe_sensitivity_field": [_vp, _vp, _i, _i, _i, _f, _f, _vp, _sz, _vp],
+    "safe_partition_indicator": [_vp, _i, _vp, _i, _i, _vp],
+    "safe_sw_cfg": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _vp],
 }
-_RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_attn_workspace_bytes": _sz,
+_RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_attn_workspace_bytes": _sz, "safe_sensitivity_workspace_bytes": _sz,
              "safe_status_string": ctypes.c_char_p}
 
 
@@ -275,3 +279,50 @@ def device_status() -> int:
 def selftest_wait_timeout(limit_ns: int = 1_000_000) -> None:
     """Launch the bounded-wait self-test (see safe_selftest_wait_timeout)."""
     _check("safe_selftest_wait_timeout", lib().safe_selftest_wait_timeout(int(limit_ns), _stream()))
+
+
+def sensitivity_workspace_bytes(B: int, N: int) -> int:
+    return int(lib().safe_sensitivity_workspace_bytes(B, N))
+
+
+def sensitivity_field(scores, grid_h: int, grid_w: int, sigma: float, truncate: float = 4.0, out=None, ws=None):
+    """s = Norm(G_sigma * s~) of Eq. (11) on the grid_h x grid_w latent grid
+    (row-major tokens), per sample: [B, N] fp32 -> [B, N] fp32 in [0, 1]."""
+    _need(scores, "scores", torch.float32, 2)
+    B, N = scores.shape
+    out = torch.empty_like(scores) if out is None else out
+    nbytes = sensitivity_workspace_bytes(B, N)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=scores.device)
+    _check("safe_sensitivity_field", lib().safe_sensitivity_field(
+        _p(scores), _p(out), B, grid_h, grid_w, float(sigma), float(truncate), _p(ws), ws.numel(), _stream()))
+    return out
+
+
+def partition_indicator(S, N: int, out=None):
+    """Binary field of the SW-CFG binary variant: 1 on S, 0 on C ([B, N] fp32)."""
+    _need(S, "S", torch.int32, 2)
+    B, k = S.shape
+    out = torch.empty((B, N), dtype=torch.float32, device=S.device) if out is None else out
+    _check("safe_partition_indicator", lib().safe_partition_indicator(_p(S), k, _p(out), B, N, _stream()))
+    return out
+
+
+_CFG_DTYPES = {torch.float32: 2, torch.bfloat16: 4}
+
+
+def sw_cfg(f_c, f_u, s, gamma_ctx: float, gamma_sens: float, out=None):
+    """Sensitivity-weighted CFG, Eq. (20), (21): f_u + gamma_i (f_c - f_u),
+    gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) s_i. f_c, f_u [B, N, C]
+    (fp32 or bf16), s [B, N] fp32; out may be f_c or f_u (in place)."""
+    if f_c.dtype not in _CFG_DTYPES or f_u.dtype != f_c.dtype:
+        raise ValueError("f_c and f_u must both be float32 or both bfloat16")
+    _need(f_c, "f_c", f_c.dtype, 3)
+    _need(f_u, "f_u", f_c.dtype, 3)
+    _need(s, "s", torch.float32, 2)
+    B, N, C = f_c.shape
+    out = torch.empty_like(f_c) if out is None else out
+    _check("safe_sw_cfg", lib().safe_sw_cfg(_p(f_c), _p(f_u), _p(s), _p(out), _CFG_DTYPES[f_c.dtype], B, N, C,
+                                            float(gamma_ctx), float(gamma_sens), _stream()))
+    return out
+

@@ -47,7 +47,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.safe_abi_version() == 2
+    assert lib.safe_abi_version() == 3
     assert lib.safe_status_string(0) == b"ok"
     assert lib.safe_status_string(1) == b"invalid argument"
     assert lib.safe_status_string(99) == b"unknown status"
@@ -116,3 +116,30 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros((1, 16, 1, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.attn_self(x, x, x)
+
+
+def test_guidance_entry_points_validate_on_host(lib):
+    null = None
+    fake = ctypes.c_void_p(0x10000)
+    other = ctypes.c_void_p(0x20000)
+    ws_ok = lib.safe_sensitivity_workspace_bytes(2, 64 * 64)
+    assert ws_ok == 2 * 4096 * 4 + 256  # row-pass field + min/max keys, each 256-byte aligned
+    assert lib.safe_sensitivity_workspace_bytes(0, 5) == 0
+    # sensitivity field: aliasing, negative sigma, bad truncate, short / misaligned workspace, radius > 128
+    assert lib.safe_sensitivity_field(fake, fake, 2, 64, 64, 1.0, 4.0, other, ws_ok, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 64, 64, -1.0, 4.0, fake, ws_ok, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 64, 64, 1.0, 0.0, fake, ws_ok, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 64, 64, float("inf"), 4.0, fake, ws_ok, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 64, 64, 1.0, 4.0, fake, ws_ok - 4, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 64, 64, 1.0, 4.0, ctypes.c_void_p(0x10080), ws_ok, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 0, 64, 1.0, 4.0, fake, ws_ok, null) == 1
+    assert lib.safe_sensitivity_field(fake, other, 2, 64, 64, 32.2, 4.0, fake, ws_ok, null) == 2  # r = 129
+    # partition indicator: k out of range
+    assert lib.safe_partition_indicator(fake, 0, other, 1, 16, null) == 1
+    assert lib.safe_partition_indicator(fake, 17, other, 1, 16, null) == 1
+    # SW-CFG: dtype fp16 unsupported, misaligned fp32, non-finite scale, empty
+    assert lib.safe_sw_cfg(fake, fake, fake, fake, 3, 1, 16, 4, 1.0, 2.0, null) == 2
+    assert lib.safe_sw_cfg(ctypes.c_void_p(0x10002), fake, fake, fake, 2, 1, 16, 4, 1.0, 2.0, null) == 1
+    assert lib.safe_sw_cfg(fake, fake, fake, fake, 2, 1, 16, 4, float("nan"), 2.0, null) == 1
+    assert lib.safe_sw_cfg(fake, fake, fake, fake, 4, 1, 16, 0, 1.0, 2.0, null) == 1
+
