@@ -37,9 +37,6 @@ from mask_free_b200 import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s + ms/call (dense, SRSU) at N=4096/25600; % bf16 tensor peak"
 WORKLOAD = "2560^2-equivalent SRSU step: B=2, H=24, d=96, N=25600, M=128 (len U[8,128]), k=6400 (0.25N)"
-# classify 3, self 1 (+1 workspace-counter reset when the key split is used), cross 1, pcsp 3 (scores,
-# head sum, top-k), scatter 1, srsu 1 (+1), cross(S) 1
-LAUNCHES_PER_STEP = 11
 
 
 def max_over_ranks(ms: float, dist=None, device=None) -> float:
@@ -185,6 +182,12 @@ class Step:
         self.ws_srsu = torch.empty(max(256, ops.attn_workspace_bytes(B, k, N, H, d)), dtype=torch.uint8, device=dev)
         self.Kc, self.Vc = inp["Kc"].clone(), inp["Vc"].clone()
         self.events = []
+        # library kernels per step: classify 3 (init, rows, verdict); dense 1
+        # (+1 merge when the last wave is split along the keys); cross with
+        # PCSP 3 (cross, head sum, top-k); scatter 1; SRSU 1 (+1 merge);
+        # cross on S 1
+        self.launches = 3 + 1 + (ops.attn_workspace_bytes(B, N, N, H, d) > 0) + 3 + 1 + 1 + \
+            (ops.attn_workspace_bytes(B, k, N, H, d) > 0) + 1
 
     def __call__(self, timed=False):
         o, i = self.ops, self.inp
@@ -197,9 +200,10 @@ class Step:
         o.attn_self(i["Q"], i["K"], i["V"], out=self.O, ws=self.ws_self)
         if timed:
             ev[1].record()
-        o.attn_cross(i["Q"], i["Ky"], i["Vy"], i["valid_len"], out=self.Ox)
-        o.pcsp_topk(i["Q"], i["Ky"], i["valid_len"], i["w"], scores=self.scores, k=self.s.k, S=self.S, C=self.C,
-                    ws=self.ws)
+        # cross-attention and, from the same probabilities (Eq. (9)), the PCSP
+        # scores and the top-k split
+        o.attn_cross_pcsp(i["Q"], i["Ky"], i["Vy"], i["valid_len"], i["w"], out=self.Ox, scores=self.scores,
+                          k=self.s.k, S=self.S, C=self.C, ws=self.ws)
         o.ctx_cache_scatter(i["K"], i["V"], self.S, self.Kc, self.Vc, src_compact=False)
         if timed:
             ev[2].record()
@@ -293,6 +297,11 @@ def kernel_table(dev, pk):
             t_p = time_kernel(lambda: ops.pcsp_topk(inp["Q"], inp["Ky"], inp["valid_len"], inp["w"], scores=sc, ws=ws))
             pb = 2 * s.B * s.N * s.H * s.d + 4 * s.B * s.H * s.N * 2 + 4 * s.B * s.N
             out["pcsp_scores"] = {"ms": t_p, "gbs": pb / t_p / 1e6, "pct_hbm": 100 * pb / t_p / 1e6 / pk["hbm"]}
+            t_xp = time_kernel(lambda: ops.attn_cross_pcsp(inp["Q"], inp["Ky"], inp["Vy"], inp["valid_len"], inp["w"],
+                                                           out=Ox, scores=sc, ws=ws))
+            xpb = xbytes + 4 * s.B * s.H * s.N * 2 + 4 * s.B * s.N
+            out["cross_with_pcsp"] = {"ms": t_xp, "gbs": xpb / t_xp / 1e6, "pct_hbm": 100 * xpb / t_xp / 1e6 / pk["hbm"],
+                                      "vs_separate_calls": (t_x + t_p) / t_xp}
             Sk = torch.empty((s.B, k), dtype=torch.int32, device=dev)
             Ck = torch.empty((s.B, s.N - k), dtype=torch.int32, device=dev)
             t_t = time_kernel(lambda: ops.topk_partition(sc, k, S=Sk, C=Ck))
@@ -472,6 +481,7 @@ def main():
                              f"frac of burst {achieved / pk['bf16']:.3f}"}
     kernels = {"dense_in_step_ms": dense_ms, "srsu_in_step_ms": statistics.mean(srsu_list),
                "srsu_in_step_tflops": f_srsu / (statistics.mean(srsu_list) * 1e-3) / 1e12}
+    launches = step.launches * args.steps
     del step
     torch.cuda.empty_cache()
     if not args.no_kernel_table:
@@ -488,7 +498,7 @@ def main():
                        "l2": "inputs exceed L2 (236 MB per image tensor); no flush",
                        "flops_per_step": f_step},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clk.summary(), "kernels": kernels,
+            "gpu_launches": launches, "clocks": clk.summary(), "kernels": kernels,
         }), flush=True)
     if dist is not None:
         dist.barrier()

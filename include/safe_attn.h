@@ -177,6 +177,19 @@ safe_status safe_pcsp_topk_noalloc(const void* Q, const void* Ky, const int32_t*
                                    int32_t* S, int32_t* C, void* stream);
 
 /*
+ * Cross-attention and PCSP scores in one pass over the queries (the scores
+ * of Eq. (10) are taken from the probabilities of the cross-attention call
+ * itself, Eq. (9)): O exactly as safe_attn_cross with q_idx = NULL, and
+ * scores / S / C exactly as safe_pcsp_topk with the same Q, Ky, valid_len,
+ * w, accumulate and k (same arithmetic, bit-identical results).
+ *  Arguments as those two calls; ws sized safe_pcsp_workspace_bytes(B, N, H).
+ */
+safe_status safe_attn_cross_pcsp(const void* Q, const void* Ky, const void* Vy, const int32_t* valid_len,
+                                 const float* w, void* O, int B, int N, int M, int H, int d, float scale,
+                                 float* scores, int accumulate, int k, int32_t* S, int32_t* C, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/*
  * Top-k partition of Eq. (12) on given scores: S[b] = the k tokens with the
  * largest score, ordered by (score descending, index ascending) so ties go to
  * the lower index; -0.0 ranks as +0.0; C[b] = the other N-k tokens. Both are

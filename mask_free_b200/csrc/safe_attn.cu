@@ -488,6 +488,34 @@ safe_status safe_pcsp_topk(const void* Q, const void* Ky, const int32_t* valid_l
   return SAFE_OK;
 }
 
+safe_status safe_attn_cross_pcsp(const void* Q, const void* Ky, const void* Vy, const int32_t* valid_len,
+                                 const float* w, void* O, int B, int N, int M, int H, int d, float scale,
+                                 float* scores, int accumulate, int k, int32_t* S, int32_t* C, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (!aligned16(Q) || !aligned16(Ky) || !aligned16(Vy) || !aligned16(O) || valid_len == nullptr || scores == nullptr)
+    return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || M < 1 || !std::isfinite(scale) || k < 0 || k > N || (k > 0 && S == nullptr))
+    return SAFE_ERR_INVALID_ARG;
+  if (!supported_d(d) || M > 256) return SAFE_ERR_UNSUPPORTED;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < safe_pcsp_workspace_bytes(B, N, H))
+    return SAFE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  CrossParams p;
+  // one pass over the queries: the output rows and, from the same
+  // probabilities, the per-head score partials
+  safe_status st = fill_cross(p, Q, nullptr, N, Ky, Vy, valid_len, w, O, static_cast<float*>(ws), B, N, M, H, d,
+                              scale);
+  if (st != SAFE_OK) return st;
+  st = dispatch_cross(d, p, s);
+  if (st != SAFE_OK) return st;
+  pcsp_reduce_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(static_cast<const float*>(ws), scores, B, H, N,
+                                                              accumulate ? 1 : 0);
+  st = launch_status();
+  if (st != SAFE_OK) return st;
+  if (k > 0) return safe_topk_partition(scores, B, N, k, S, C, stream);
+  return SAFE_OK;
+}
+
 safe_status safe_pcsp_topk_noalloc(const void* Q, const void* Ky, const int32_t* valid_len, const float* w, int B,
                                    int N, int M, int H, int d, float scale, float* scores, int accumulate, int k,
                                    int32_t* S, int32_t* C, void* stream) {

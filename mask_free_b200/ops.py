@@ -41,6 +41,8 @@ _SIGS = {
     "safe_status_string": [_i],
     "safe_selftest_wait_timeout": [ctypes.c_uint64, _vp],
     "safe_pcsp_topk_noalloc": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
+    "safe_attn_cross_pcsp": [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp,
+                             _sz, _vp],
     "safe_sensitivity_workspace_bytes": [_i, _i],
     "safe_sensitivity_field": [_vp, _vp, _i, _i, _i, _f, _f, _vp, _sz, _vp],
     "safe_partition_indicator": [_vp, _i, _vp, _i, _i, _vp],
@@ -220,6 +222,33 @@ def pcsp_topk(Q, Ky, valid_len, w=None, scores=None, accumulate=False, k=0, scal
         _p(Q), _p(Ky), _p(valid_len), _p(w), B, N, M, H, d, _scale(d, scale), _p(scores), 1 if accumulate else 0, k,
         _p(S), _p(C), _p(ws), ws.numel() if ws is not None else 0, _stream()))
     return scores, S, C
+
+
+def attn_cross_pcsp(Q, Ky, Vy, valid_len, w=None, out=None, scores=None, accumulate=False, k=0, scale=None, S=None,
+                    C=None, ws=None):
+    """Cross-attention (Eq. (4)) and the PCSP scores of Eq. (10) from the same
+    probabilities, in one pass over Q; with k > 0 also the top-k split
+    (Eq. (12)). Returns (O, scores, S, C)."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(Ky, "Ky", torch.bfloat16, 4)
+    _need(Vy, "Vy", torch.bfloat16, 4)
+    _need(valid_len, "valid_len", torch.int32, 1)
+    if w is not None:
+        _need(w, "w", torch.float32, 2)
+    B, N, H, d = Q.shape
+    M = Ky.shape[1]
+    out = torch.empty_like(Q) if out is None else out
+    if scores is None:
+        scores = torch.zeros((B, N), dtype=torch.float32, device=Q.device)
+    if k > 0:
+        S = torch.empty((B, k), dtype=torch.int32, device=Q.device) if S is None else S
+        C = torch.empty((B, N - k), dtype=torch.int32, device=Q.device) if C is None else C
+    if ws is None:
+        ws = torch.empty(max(pcsp_workspace_bytes(B, N, H), 256), dtype=torch.uint8, device=Q.device)
+    _check("safe_attn_cross_pcsp", lib().safe_attn_cross_pcsp(
+        _p(Q), _p(Ky), _p(Vy), _p(valid_len), _p(w), _p(out), B, N, M, H, d, _scale(d, scale), _p(scores),
+        1 if accumulate else 0, k, _p(S), _p(C), _p(ws), ws.numel(), _stream()))
+    return out, scores, S, C
 
 
 def topk_partition(scores, k, S=None, C=None, with_c=True):

@@ -143,3 +143,15 @@ def test_guidance_entry_points_validate_on_host(lib):
     assert lib.safe_sw_cfg(fake, fake, fake, fake, 2, 1, 16, 4, float("nan"), 2.0, null) == 1
     assert lib.safe_sw_cfg(fake, fake, fake, fake, 4, 1, 16, 0, 1.0, 2.0, null) == 1
 
+
+def test_fused_cross_pcsp_validates_on_host(lib):
+    null = None
+    fake = ctypes.c_void_p(0x10000)
+    ws_ok = lib.safe_pcsp_workspace_bytes(1, 16, 1)
+    args = lambda M, k, ws, wsb: (fake, fake, fake, fake, null, fake, 1, 16, M, 1, 96, 1.0, fake, 0, k, fake, null,
+                                  ws, wsb, null)
+    assert lib.safe_attn_cross_pcsp(*args(16, 4, null, 0)) == 1             # no workspace
+    assert lib.safe_attn_cross_pcsp(*args(16, 4, fake, ws_ok - 4)) == 1     # short workspace
+    assert lib.safe_attn_cross_pcsp(*args(16, 17, fake, ws_ok)) == 1        # k > N
+    assert lib.safe_attn_cross_pcsp(*args(257, 4, fake, ws_ok)) == 2        # M > 256
+

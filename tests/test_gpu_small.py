@@ -263,6 +263,25 @@ def test_pcsp_scores_parity_uniform_and_accumulate():
     assert torch.equal(sp, sc)
 
 
+def test_fused_cross_pcsp_equals_separate_calls_bitwise():
+    B, N, M, H, d, k = 2, 1000, 128, 3, 96, 301
+    Q = rnd_bf16((B, N, H, d), 51)
+    Ky, Vy = rnd_bf16((B, M, H, d), 52), rnd_bf16((B, M, H, d), 53)
+    lens = torch.tensor([29, 128], dtype=torch.int32, device=DEV)
+    w = synth.content_weights(lens.cpu(), M, 54).to(DEV)
+    Qd, Kd, Vd = Q.to(DEV), Ky.to(DEV), Vy.to(DEV)
+    O_sep = ops.attn_cross(Qd, Kd, Vd, lens)
+    sc_sep, S_sep, C_sep = ops.pcsp_topk(Qd, Kd, lens, w, k=k)
+    O_f, sc_f, S_f, C_f = ops.attn_cross_pcsp(Qd, Kd, Vd, lens, w, k=k)
+    assert torch.equal(O_f, O_sep) and torch.equal(sc_f, sc_sep)
+    assert torch.equal(S_f, S_sep) and torch.equal(C_f, C_sep)
+    # and against the oracle
+    ref = O.pcsp_scores(to64(Q), to64(Ky), [29, 128], w.cpu().numpy().astype(np.float64), 1 / math.sqrt(d))
+    np.testing.assert_allclose(sc_f.cpu().numpy(), ref, rtol=2e-5, atol=1e-8)
+    assert_attn_close(O_f, O.cross_attention(to64(Q), to64(Ky), to64(Vy), [29, 128], 1 / math.sqrt(d)), "fused")
+    assert ops.device_status() == 0
+
+
 def _valid_topk(S, C, scores64, k, tol):
     S, C = S.cpu().numpy(), C.cpu().numpy()
     for b in range(S.shape[0]):
