@@ -449,27 +449,52 @@ def main():
     ms_step = ms_total / args.steps
     value = job_throughput(world, f_step, ms_step)
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, the step, D2H of its outputs
+    # end to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory and its results back. Two device
+    # buffer sets and two copy streams let the copies of one step overlap
+    # the compute of its neighbours; each step still starts only after its
+    # own inputs have arrived, and the clock stops after the last results
+    # are on the host. (The all-valid attention mask is a device-resident
+    # tensor of the model, shared by both sets, and is not re-sent.)
     host = {n: inp[n].cpu().pin_memory() for n in ("Q", "K", "V", "Ky", "Vy", "valid_len", "w")}
-    outs = [step.O, step.Ox, step.Os, step.Osx, step.S]
-    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    inp2 = {n: (t if n == "mask" else t.clone()) for n, t in inp.items()}
+    sets = [(inp, step), (inp2, Step(s, inp2, dev))]
+    outs = [[st.O, st.Ox, st.Os, st.Osx, st.S] for _, st in sets]
+    host_out = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs[0]] for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    comp, s_in, s_out = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in, ev_done, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_steps = max(2, min(args.steps, 5))
-    e0.record()
-    for _ in range(e_steps):
-        for n, t in host.items():
-            inp[n].copy_(t, non_blocking=True)
-        step()
-        for o, ho in zip(outs, host_out):
-            ho.copy_(o, non_blocking=True)
-    e1.record()
+    e_steps = max(4, min(args.steps, 10))
+    torch.cuda.synchronize()
+    e0.record(s_in)
+    for i in range(e_steps):
+        b = i % 2
+        ins, st = sets[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[b])  # step i-2 has finished reading this set
+            for n, t in host.items():
+                ins[n].copy_(t, non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        if i >= 2:
+            comp.wait_event(ev_out[b])  # step i-2's results have left this set
+        st()
+        ev_done[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            for o, ho in zip(outs[b], host_out[b]):
+                ho.copy_(o, non_blocking=True)
+            ev_out[b].record(s_out)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / e_steps, dist, dev)
     e2e = {"value": job_throughput(world, f_step, ms_e2e), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+           "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": e_steps,
+           "overlap": "copies of step i overlap the compute of steps i-1 / i+1 (two buffer sets)"}
+    del sets, inp2, outs
 
     dense_list, srsu_list = step.launch_times()
     dense_ms = statistics.mean(dense_list)
