@@ -279,6 +279,25 @@ def kernel_table(dev, pk):
         out[f"srsu_{tag}_k{k}"] = {"ms": t_s, "tflops": srsu_f / t_s / 1e9,
                                    "pct_bf16_burst": 100 * srsu_f / t_s / 1e9 / pk["bf16"],
                                    "pct_bf16_sustained": 100 * srsu_f / t_s / 1e9 / pk["bf16_sustained"]}
+        # context only (the pages' mask-induced dispatch tax, on this machine):
+        # torch's own SDPA on the same tensors without a mask and with the
+        # all-valid boolean mask that the classifier certifies removable
+        # (fused backends only: the unfused one would materialise N x N scores)
+        try:
+            import torch.nn.functional as F
+            from torch.nn.attention import SDPBackend, sdpa_kernel
+            qt, kt, vt = (inp[n].transpose(1, 2) for n in ("Q", "K", "V"))
+            with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION, SDPBackend.CUDNN_ATTENTION]):
+                t_free = time_kernel(lambda: F.scaled_dot_product_attention(qt, kt, vt), reps=3, warm=1)
+                t_mask = time_kernel(lambda: F.scaled_dot_product_attention(qt, kt, vt, attn_mask=inp["mask"]),
+                                     reps=3, warm=1)
+            out[f"torch_sdpa_context_N{s.N}"] = {
+                "mask_free_ms": t_free, "all_valid_bool_mask_ms": t_mask, "masked_over_mask_free": t_mask / t_free,
+                "ours_dense_ms": t_d}
+            del qt, kt, vt
+        except Exception as e:  # context only: record why it could not run
+            out[f"torch_sdpa_context_N{s.N}"] = {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
+        torch.cuda.synchronize()
         xbytes = 2 * 2 * s.B * s.N * s.H * s.d + 2 * 2 * s.B * s.M * s.H * s.d
         out[f"cross_{tag}"] = {"ms": t_x, "gbs": xbytes / t_x / 1e6, "pct_hbm": 100 * xbytes / t_x / 1e6 / pk["hbm"],
                                "tflops": cross_f / t_x / 1e9}
