@@ -11,12 +11,11 @@
 //               S = Q Ky^T (N = Lp = ceil32(valid_len)) into TMEM, then
 //               O = P Vy with P read from TMEM;
 //   warp 3      output store: the bf16 O tile, staged by the warpgroup in
-//               the slot its query tile came from, leaves by TMA store, and
-//               the slot returns to the producer;
+//               shared memory, leaves by TMA store;
 //   warps 4..11 two softmax warpgroups, one query row per thread: max over
-//               the valid keys, p = 2^(s*scale*log2(e) - max), l = sum p,
+//               the keys, p = 2^(s*scale*log2(e) - max), l = sum p,
 //               score = sum_j w_j p_j / l (the PCSP partial of this head),
-//               P (bf16) back into TMEM; after P V, O / l into the slot.
+//               P (bf16) into TMEM; after P V, O / l into the staging buffer.
 // Before the first tile the text key / value rows [0, Lp) are copied into the
 // swizzled layouts the tensor core reads, zeros for rows >= valid_len
 // (padding rows are never read, so they may hold any bytes). The padding
@@ -25,11 +24,12 @@
 // -inf for padding keys, so S arrives with -inf in every padding column and
 // the softmax has no mask to apply.
 //
-// TMEM (512 columns): warpgroup g owns [256g, 256g + 256): S in [0, Lp), P
-// (bf16 pairs) over its first Lp/2 columns, O in [128, 128 + D). For
-// Lp <= 128 the next S of a warpgroup only waits for the previous P V
-// product; for Lp > 128 it overlaps O and waits for the previous output to
-// be read.
+// Two TMEM layouts (512 columns; see cross_sep_p below): for D <= 96 and
+// M <= 128, S0, S1, O0, O1 and one P buffer shared by the warpgroups in
+// alternation, with S released as soon as it is loaded and the output
+// staged in two buffers of its own; otherwise warpgroup g owns
+// [256g, 256g + 256) (S at 0 with P over it, O at 128) and stages its output
+// in the slot its query tile came from.
 #pragma once
 
 #include <type_traits>
