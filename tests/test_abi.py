@@ -155,3 +155,11 @@ def test_fused_cross_pcsp_validates_on_host(lib):
     assert lib.safe_attn_cross_pcsp(*args(16, 17, fake, ws_ok)) == 1        # k > N
     assert lib.safe_attn_cross_pcsp(*args(257, 4, fake, ws_ok)) == 2        # M > 256
 
+
+
+def test_graft_entry_build_loads_the_library():
+    # the build entry point compiles (if needed), loads the library and
+    # checks the ABI version it was written against
+    import __graft_entry__ as g
+    g.build()
+    assert ops.abi_version() == 3
