@@ -100,10 +100,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, log_dir: str = None):
+        import tempfile
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"clocks_rank{device_index}.csv")
 
     def __enter__(self):
         try:
@@ -146,16 +147,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def make_step_inputs(config: int, dev):
-    s = synth.CONFIGS[config]
-    g = torch.Generator(device=dev).manual_seed(1000 * config)
+def make_step_inputs(workload: str, dev):
+    s = synth.WORKLOADS[workload]
+    g = torch.Generator(device=dev).manual_seed(1000 * s.seed_id)
 
     def bf(rows):
         return torch.randn((s.B, rows, s.H, s.d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
 
-    lens = synth.uniform_lengths(s.B, s.len_lo, s.len_hi, synth.seed_for(config, synth.T_LEN))
+    lens = synth.uniform_lengths(s.B, s.len_lo, s.len_hi, synth.seed_for(s.seed_id, synth.T_LEN))
     inp = {"Q": bf(s.N), "K": bf(s.N), "V": bf(s.N), "Ky": bf(s.M), "Vy": bf(s.M),
-           "valid_len": lens.to(dev), "w": synth.content_weights(lens, s.M, synth.seed_for(config, synth.T_W)).to(dev)}
+           "valid_len": lens.to(dev), "w": synth.content_weights(lens, s.M, synth.seed_for(s.seed_id, synth.T_W)).to(dev)}
     inp["Kc"] = (inp["K"].float() + 0.05 * torch.randn(inp["K"].shape, generator=g, device=dev)).to(torch.bfloat16)
     inp["Vc"] = (inp["V"].float() + 0.05 * torch.randn(inp["V"].shape, generator=g, device=dev)).to(torch.bfloat16)
     inp["mask"] = torch.ones((s.B, 1, s.N, s.N), dtype=torch.bool, device=dev)
@@ -256,9 +257,9 @@ def kernel_table(dev, pk):
     memory-bound kernels' GB/s at N = 25600, and the SRSU |S|/N sweep."""
     from mask_free_b200 import ops
     out = {"timing": "device ms per call: CUDA-graph replay of 20 back-to-back calls"}
-    for config in (2, 4):
-        s, inp, lsum = make_step_inputs(config, dev)
-        if config == 2:
+    for workload in ("n4096", "n25600"):
+        s, inp, lsum = make_step_inputs(workload, dev)
+        if workload == "n4096":
             k = s.k
         else:
             k = s.k
@@ -301,7 +302,7 @@ def kernel_table(dev, pk):
         xbytes = 2 * 2 * s.B * s.N * s.H * s.d + 2 * 2 * s.B * s.M * s.H * s.d
         out[f"cross_{tag}"] = {"ms": t_x, "gbs": xbytes / t_x / 1e6, "pct_hbm": 100 * xbytes / t_x / 1e6 / pk["hbm"],
                                "tflops": cross_f / t_x / 1e9}
-        if config == 4:
+        if workload == "n25600":
             # memory-bound kernels
             cls = torch.empty(3, dtype=torch.int64, device=dev)
             t_c = time_kernel(lambda: ops.mask_classify(inp["mask"], sync=False, result=cls))
@@ -365,7 +366,7 @@ class OracleSample:
     pairs, against all keys."""
 
     def __init__(self):
-        s = synth.CONFIGS[4]
+        s = synth.WORKLOADS["n25600"]
         rng = np.random.default_rng(0)
         shape = (s.B, s.N, s.H, s.d)
         self.s = s
@@ -420,6 +421,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-kernel-table", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None, help="directory for the raw clock samples (default: a temp dir)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -443,7 +445,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     pk = peaks()
-    s, inp, lsum = make_step_inputs(4, dev)
+    s, inp, lsum = make_step_inputs("n25600", dev)
     step = Step(s, inp, dev)
     f_dense, f_srsu, f_cross, f_cross_s = flops(s, lsum, s.k)
     f_step = f_dense + f_srsu + f_cross + f_cross_s
@@ -455,7 +457,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, args.clock_log) as clk:
         t0.record()
         for _ in range(args.steps):
             step(timed=True)

@@ -1,10 +1,10 @@
 """Run one kernel of the hot path a few times on one workload, for profilers.
 
-    python -m mask_free_b200.profile_case --kernel self --config 2 --launches 3
+    python -m mask_free_b200.profile_case --kernel self --workload n4096 --launches 3
 
 Kernels: self, srsu, cross, pcsp, topk, scatter, classify. Inputs are
 generated on the device (standard normals in bf16, like the benchmark), so
-the process holds only the tensors of that one call (config 2: ~0.2 GB).
+the process holds only the tensors of that one call (n4096: ~0.2 GB).
 """
 
 from __future__ import annotations
@@ -20,12 +20,12 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", required=True, choices=["self", "srsu", "cross", "pcsp", "topk", "scatter",
                                                         "classify"])
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--workload", default="n4096", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--launches", type=int, default=3)
     a = ap.parse_args()
-    s = synth.CONFIGS[a.config]
+    s = synth.WORKLOADS[a.workload]
     dev = torch.device("cuda")
-    g = torch.Generator(device=dev).manual_seed(a.config)
+    g = torch.Generator(device=dev).manual_seed(s.seed_id)
 
     def bf(rows):
         return torch.randn((s.B, rows, s.H, s.d), generator=g, device=dev).to(torch.bfloat16)
@@ -56,7 +56,7 @@ def main():
             ops.mask_classify(m)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
-    print("ok", a.kernel, a.config, a.launches)
+    print("ok", a.kernel, a.workload, a.launches)
 
 
 if __name__ == "__main__":

@@ -8,7 +8,8 @@ exactly by the oracle).
 Recipe (workload shapes of the paper's Lumina-Next runs at 1024^2, 2560^2
 and 3072^2, with a 16x spatial reduction from pixels to latent tokens):
   * Q, K, V, K_y, V_y: fp32 standard normals from numpy PCG64(seed), rounded
-    to bf16 with round-to-nearest-even; seed = 1000 * config + tensor id.
+    to bf16 with round-to-nearest-even; seed = 1000 * (workload seed id) +
+    100 * call + tensor id.
   * text valid lengths: uniform integers in [lo, hi] per sample.
   * content weights w: U(0, 1) on valid keys, 0 on padding, normalised to
     sum 1 per sample in fp64, stored as fp32.
@@ -26,8 +27,8 @@ import torch
 T_Q, T_K, T_V, T_KY, T_VY, T_LEN, T_W, T_DK, T_DV, T_MASK = range(10)
 
 
-def seed_for(config: int, tensor_id: int, call: int = 0) -> int:
-    return 1000 * config + 100 * call + tensor_id
+def seed_for(seed_id: int, tensor_id: int, call: int = 0) -> int:
+    return 1000 * seed_id + 100 * call + tensor_id
 
 
 def normal_f32(shape, seed: int) -> np.ndarray:
@@ -73,6 +74,7 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
 
 @dataclass(frozen=True)
 class Shape:
+    seed_id: int  # distinguishes the workloads' random streams
     B: int
     N: int
     H: int
@@ -83,21 +85,22 @@ class Shape:
     k: int
 
 
-# The five workloads: tiny check, 1024^2 dense block, 1024^2 SRSU step,
-# 2560^2 anchor + SRSU, 3072^2 20-call sequence.
-CONFIGS = {
-    1: Shape(B=1, N=256, H=2, d=64, M=16, len_lo=11, len_hi=11, k=64),
-    2: Shape(B=2, N=4096, H=24, d=96, M=128, len_lo=8, len_hi=128, k=1229),
-    3: Shape(B=2, N=4096, H=24, d=96, M=128, len_lo=8, len_hi=128, k=1229),
-    4: Shape(B=2, N=25600, H=24, d=96, M=128, len_lo=8, len_hi=128, k=6400),
-    5: Shape(B=2, N=36864, H=24, d=96, M=256, len_lo=16, len_hi=256, k=7373),
+# The workloads, by what they are: a tiny check; the 1024^2 (N = 4096)
+# dense block and SRSU step; the 2560^2 (N = 25600) anchor + SRSU step; the
+# 3072^2 (N = 36864) 20-call anchor / SRSU sequence.
+WORKLOADS = {
+    "tiny": Shape(seed_id=1, B=1, N=256, H=2, d=64, M=16, len_lo=11, len_hi=11, k=64),
+    "n4096": Shape(seed_id=2, B=2, N=4096, H=24, d=96, M=128, len_lo=8, len_hi=128, k=1229),
+    "n4096_srsu": Shape(seed_id=3, B=2, N=4096, H=24, d=96, M=128, len_lo=8, len_hi=128, k=1229),
+    "n25600": Shape(seed_id=4, B=2, N=25600, H=24, d=96, M=128, len_lo=8, len_hi=128, k=6400),
+    "n36864_seq": Shape(seed_id=5, B=2, N=36864, H=24, d=96, M=256, len_lo=16, len_hi=256, k=7373),
 }
 
 
-def make_inputs(config: int, shape: Shape = None, call: int = 0, drift_std: float = 0.05):
-    """All tensors of one hot-path step for `config` (CPU, bf16 / int32 / fp32)."""
-    s = shape or CONFIGS[config]
-    c = config
+def make_inputs(workload: str, shape: Shape = None, call: int = 0, drift_std: float = 0.05):
+    """All tensors of one hot-path step of `workload` (CPU, bf16 / int32 / fp32)."""
+    s = shape or WORKLOADS[workload]
+    c = WORKLOADS[workload].seed_id
     inp = {
         "Q": normal_bf16((s.B, s.N, s.H, s.d), seed_for(c, T_Q, call)),
         "K": normal_bf16((s.B, s.N, s.H, s.d), seed_for(c, T_K, call)),
@@ -113,7 +116,7 @@ def make_inputs(config: int, shape: Shape = None, call: int = 0, drift_std: floa
 
 
 def sample_rows(N: int, count: int, seed: int) -> np.ndarray:
-    """Sorted distinct query rows drawn uniformly (for large-config parity)."""
+    """Sorted distinct query rows drawn uniformly (for sampled parity at large N)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     return np.sort(rng.choice(N, size=min(count, N), replace=False))
 

@@ -19,7 +19,7 @@ Layouts (shared with the CUDA path only through the test harness):
   scores                     [B, N]
   S, C                       [B, k], [B, N-k] int, each strictly ascending
 
-Readings of the paper where it is silent (each is listed in the design doc):
+Readings of the paper where it is silent:
   * the padding mask m_text keeps a prefix of valid keys (right padding);
   * scores are kept per sample b (Eq. (10) has no batch index);
   * top-k ties go to the lower token index; -0.0 is treated as +0.0;

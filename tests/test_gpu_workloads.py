@@ -1,9 +1,9 @@
-"""GPU parity on the five workloads (Lumina-Next-scale shapes).
+"""GPU parity on the Lumina-Next-scale workloads.
 
-configs 2/3 (N = 4096): full comparison of every output;
-configs 4/5 (N = 25600 / 36864): 512 seeded sampled query rows per head for
-the attention outputs, whole-buffer bitwise checks for the cache, and the
-20-call anchor / SRSU sequence of config 5 replayed by the oracle.
+N = 4096 (dense block, SRSU step): full comparison of every output;
+N = 25600 / 36864: 512 seeded sampled query rows per head for the attention
+outputs, whole-buffer bitwise checks for the cache, and the 20-call anchor /
+SRSU sequence at N = 36864 replayed by the oracle.
 The partition S used by the GPU calls is the oracle's own (from its fp64 PCSP
 scores); the GPU's PCSP split is checked separately for validity.
 """
@@ -30,9 +30,9 @@ def _status_clean():
     assert ops.device_status() == 0
 
 
-def load(config):
-    s = synth.CONFIGS[config]
-    inp = synth.make_inputs(config)
+def load(workload):
+    s = synth.WORKLOADS[workload]
+    inp = synth.make_inputs(workload)
     host64 = {n: synth.bf16_to_f64(inp[n]) for n in ("Q", "K", "V", "Ky", "Vy", "Kc", "Vc")}
     dev = {n: v.to(DEV) for n, v in inp.items()}
     return s, inp, host64, dev
@@ -58,16 +58,16 @@ def check_gpu_partition(s, dev, ref_scores):
         assert ref_scores[b][sel].min() >= ref_scores[b][~sel].max() - tol
 
 
-@pytest.mark.parametrize("config", [2, 3])
-def test_config_n4096_full(config):
-    s, inp, h, d = load(config)
+@pytest.mark.parametrize("workload", ["n4096", "n4096_srsu"])
+def test_n4096_full(workload):
+    s, inp, h, d = load(workload)
     scale = 1 / math.sqrt(s.d)
     lens = inp["valid_len"].numpy()
-    if config == 2:
+    if workload == "n4096":
         assert_attn_close(ops.attn_self(d["Q"], d["K"], d["V"]), O.attention(h["Q"], h["K"], h["V"], scale),
-                          "cfg2 self")
+                          "n4096 self")
         assert_attn_close(ops.attn_cross(d["Q"], d["Ky"], d["Vy"], d["valid_len"]),
-                          O.cross_attention(h["Q"], h["Ky"], h["Vy"], lens, scale), "cfg2 cross")
+                          O.cross_attention(h["Q"], h["Ky"], h["Vy"], lens, scale), "n4096 cross")
         mask = torch.ones((s.B, 1, s.N, s.N), dtype=torch.bool, device=DEV)
         assert ops.mask_classify(mask) == (1, 0, -1)
         return
@@ -86,24 +86,24 @@ def test_config_n4096_full(config):
     assert np.array_equal(synth.bf16_bits(Vc.cpu()).reshape(shape), Vc_ref)
     out = ops.srsu_attn(d["Q"], S_dev, Kc, Vc)
     assert_attn_close(out, O.srsu_attention(h["Q"], S_ref, O.bf16_bits_to_f64(Kc_ref), O.bf16_bits_to_f64(Vc_ref),
-                                            scale), "cfg3 srsu")
+                                            scale), "n4096 srsu")
     outx = ops.attn_cross(d["Q"], d["Ky"], d["Vy"], d["valid_len"], q_idx=S_dev)
-    assert_attn_close(outx, O.cross_attention(h["Q"], h["Ky"], h["Vy"], lens, scale, q_rows=S_ref), "cfg3 cross S")
+    assert_attn_close(outx, O.cross_attention(h["Q"], h["Ky"], h["Vy"], lens, scale, q_rows=S_ref), "n4096 cross S")
 
 
-def test_config4_n25600_sampled():
-    s, inp, h, d = load(4)
+def test_n25600_sampled():
+    s, inp, h, d = load("n25600")
     scale = 1 / math.sqrt(s.d)
     lens = inp["valid_len"].numpy()
     rows = synth.sample_rows(s.N, SAMPLE, seed=4004)
     # dense anchor self-attention
     out = ops.attn_self(d["Q"], d["K"], d["V"])
-    assert_attn_close(out[:, rows], O.attention(h["Q"], h["K"], h["V"], scale, q_rows=rows), "cfg4 self")
+    assert_attn_close(out[:, rows], O.attention(h["Q"], h["K"], h["V"], scale, q_rows=rows), "n25600 self")
     del out
     # cross-attention
     outx = ops.attn_cross(d["Q"], d["Ky"], d["Vy"], d["valid_len"])
     assert_attn_close(outx[:, rows], O.cross_attention(h["Q"], h["Ky"], h["Vy"], lens, scale, q_rows=rows),
-                      "cfg4 cross")
+                      "n25600 cross")
     del outx
     # PCSP -> (oracle) partition -> scatter -> SRSU over the drifted cache
     ref_scores, S_ref, _ = oracle_partition(s, inp, h, scale)
@@ -122,16 +122,16 @@ def test_config4_n25600_sampled():
     rsel = synth.sample_rows(s.k, SAMPLE, seed=4005)
     ref = O.attention(h["Q"], O.bf16_bits_to_f64(Kc_ref), O.bf16_bits_to_f64(Vc_ref), scale,
                       q_rows=S_ref[:, rsel])
-    assert_attn_close(out[:, rsel], ref, "cfg4 srsu")
+    assert_attn_close(out[:, rsel], ref, "n25600 srsu")
 
 
-def test_config5_twenty_call_sequence():
+def test_n36864_twenty_call_sequence():
     """Anchor (dense + full refresh, Eq. (18)/(19)) at calls 0, 5, 10, 15;
     otherwise scatter of the sensitive rows + SRSU (Eq. (15)/(16)), with the
     cache updated in place. Call t uses the seeded base fields shifted along
     the tokens by (1009 t, 2003 t, 3001 t) for (Q, K, V) (exact copies)."""
-    s = synth.CONFIGS[5]
-    inp = synth.make_inputs(5)
+    s = synth.WORKLOADS["n36864_seq"]
+    inp = synth.make_inputs("n36864_seq")
     scale = 1 / math.sqrt(s.d)
     lens = inp["valid_len"].numpy()
     h64 = {n: synth.bf16_to_f64(inp[n]) for n in ("Q", "Ky")}
@@ -159,7 +159,7 @@ def test_config5_twenty_call_sequence():
             if t in (0, 15):
                 ref = O.attention(O.bf16_bits_to_f64(cur_h["Q"]), O.bf16_bits_to_f64(cur_h["K"]),
                                   O.bf16_bits_to_f64(cur_h["V"]), scale, q_rows=rows)
-                assert_attn_close(out[:, rows], ref, f"cfg5 anchor call {t}")
+                assert_attn_close(out[:, rows], ref, f"n36864 anchor call {t}")
         else:
             ops.ctx_cache_scatter(cur["K"], cur["V"], S_dev, Kc, Vc, src_compact=False)
             out = ops.srsu_attn(cur["Q"], S_dev, Kc, Vc)
@@ -168,7 +168,7 @@ def test_config5_twenty_call_sequence():
             if t in (1, 19):
                 ref = O.attention(O.bf16_bits_to_f64(cur_h["Q"]), O.bf16_bits_to_f64(cache_k),
                                   O.bf16_bits_to_f64(cache_v), scale, q_rows=S_ref[:, rsel])
-                assert_attn_close(out[:, rsel], ref, f"cfg5 srsu call {t}")
+                assert_attn_close(out[:, rsel], ref, f"n36864 srsu call {t}")
         assert np.array_equal(synth.bf16_bits(Kc.cpu()).reshape(shape), cache_k), f"K cache differs at call {t}"
         assert np.array_equal(synth.bf16_bits(Vc.cpu()).reshape(shape), cache_v), f"V cache differs at call {t}"
         del out, cur
@@ -176,4 +176,4 @@ def test_config5_twenty_call_sequence():
     Ky, Vy = d["Ky"], inp["Vy"].to(DEV)
     outx = ops.attn_cross(d["Q"], Ky, Vy, d["valid_len"])
     assert_attn_close(outx[:, rows], O.cross_attention(h64["Q"], h64["Ky"], synth.bf16_to_f64(inp["Vy"]), lens,
-                                                      scale, q_rows=rows), "cfg5 cross")
+                                                      scale, q_rows=rows), "n36864 cross")
