@@ -260,23 +260,19 @@ __global__ void __launch_bounds__(kTopkThreads) topk_partition_kernel(const floa
       if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 255u], 1);
     }
     __syncthreads();
+    // count of digit d = 255 - tid; an exclusive scan over the digits from
+    // the top gives, per digit, the number of matching keys above it: the
+    // selected digit is the one whose range [above, above + count) holds
+    // the remaining-th largest key
+    int cnt = 0;
     if (tid < 256) {
-      int s = 0;
-      for (int w = 0; w < 32; ++w) s += hist[w][tid];
-      hist[0][tid] = s;
+#pragma unroll 8
+      for (int w = 0; w < 32; ++w) cnt += hist[w][255 - tid];
     }
-    __syncthreads();
-    if (tid == 0) {
-      int cum = 0, sel = 0;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + hist[0][d] >= remaining) {
-          sel = d;
-          break;
-        }
-        cum += hist[0][d];
-      }
-      sh_prefix = prefix | (static_cast<uint32_t>(sel) << shift);
-      sh_remaining = remaining - cum;
+    const int above = block_exclusive_scan(cnt, warp_tot);
+    if (tid < 256 && above < remaining && remaining <= above + cnt) {
+      sh_prefix = prefix | (static_cast<uint32_t>(255 - tid) << shift);
+      sh_remaining = remaining - above;
     }
     __syncthreads();
     prefix = sh_prefix;
