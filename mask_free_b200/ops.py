@@ -310,6 +310,17 @@ def selftest_wait_timeout(limit_ns: int = 1_000_000) -> None:
     _check("safe_selftest_wait_timeout", lib().safe_selftest_wait_timeout(int(limit_ns), _stream()))
 
 
+def shared_partition(scores, k, sample: int = 0, B: int = None):
+    """One partition for a whole CFG pair (or batch): the top-k split of
+    Eq. (12) of one sample's scores (by default the conditional one,
+    sample 0), repeated for every sample, so that all of them update the
+    same sensitive rows. Returns S [B, k], C [B, N - k] (int32, device)."""
+    _need(scores, "scores", torch.float32, 2)
+    B = scores.shape[0] if B is None else B
+    S1, C1 = topk_partition(scores[sample:sample + 1], k)
+    return S1.expand(B, -1).contiguous(), C1.expand(B, -1).contiguous()
+
+
 def sensitivity_workspace_bytes(B: int, N: int) -> int:
     return int(lib().safe_sensitivity_workspace_bytes(B, N))
 

@@ -149,3 +149,19 @@ def test_sw_cfg_in_place_equal_scales_and_binary_variant():
     out = ops.sw_cfg(fc.to(DEV), fu.to(DEV), ind, 2.0, 9.0).cpu().numpy().astype(np.float64)
     ref = O.sw_cfg(fc.numpy(), fu.numpy(), O.partition_indicator(S.numpy(), N), 2.0, 9.0)
     np.testing.assert_allclose(out, ref, rtol=1e-6, atol=1e-6)
+
+
+def test_shared_cfg_pair_partition():
+    # the conditional sample's split, applied to both halves of the pair;
+    # bit-exact against the oracle's top-k of that sample's scores
+    N, k = 3000, 751
+    sc = torch.from_numpy(_scores(2, N, 301)).to(DEV)
+    S, C = ops.shared_partition(sc, k)
+    S_ref, C_ref = O.topk_partition(sc[:1].cpu().numpy().astype(np.float64), k)
+    for b in range(2):
+        assert np.array_equal(S[b].cpu().numpy(), S_ref[0]) and np.array_equal(C[b].cpu().numpy(), C_ref[0])
+    # SRSU of both samples then gathers the same rows
+    Sb, _ = ops.shared_partition(sc, k, sample=1)
+    S1_ref, _ = O.topk_partition(sc[1:].cpu().numpy().astype(np.float64), k)
+    assert np.array_equal(Sb[0].cpu().numpy(), S1_ref[0])
+
