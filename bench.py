@@ -312,6 +312,13 @@ def kernel_table(dev, pk):
             t_sc = time_kernel(lambda: ops.ctx_cache_scatter(inp["K"], inp["V"], S, Kc, Vc, src_compact=False))
             sb = 4 * s.B * k * s.H * s.d * 2
             out["scatter"] = {"ms": t_sc, "gbs": sb / t_sc / 1e6, "pct_hbm": 100 * sb / t_sc / 1e6 / pk["hbm"]}
+            # SRSU with K/V of S u C assembled in the kernel (no scatter pass,
+            # cache only read) against the two launches scatter + SRSU
+            t_a = time_kernel(lambda: ops.srsu_attn_assembled(inp["Q"], S, inp["K"], inp["V"], inp["Kc"], inp["Vc"],
+                                                              out=Os, ws=ws_s))
+            out[f"srsu_assembled_{tag}_k{k}"] = {
+                "ms": t_a, "tflops": srsu_f / t_a / 1e9, "pct_bf16_burst": 100 * srsu_f / t_a / 1e9 / pk["bf16"],
+                "scatter_plus_srsu_ms": t_sc + t_s, "saved_ms": t_sc + t_s - t_a}
             sc = torch.empty((s.B, s.N), dtype=torch.float32, device=dev)
             ws = torch.empty(ops.pcsp_workspace_bytes(s.B, s.N, s.H), dtype=torch.uint8, device=dev)
             t_p = time_kernel(lambda: ops.pcsp_topk(inp["Q"], inp["Ky"], inp["valid_len"], inp["w"], scores=sc, ws=ws))

@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { SAFE_BOOL = 0, SAFE_U8 = 1, SAFE_F32 = 2, SAFE_F16 = 3, SAFE_BF16 = 4 } safe_dtype;
 
-/* ABI version of this header (bumped on any signature or entry-point change): 3. */
+/* ABI version of this header (bumped on any signature or entry-point change): 4. */
 int safe_abi_version(void);
 const char* safe_status_string(int status);
 
@@ -216,6 +216,29 @@ safe_status safe_topk_partition(const float* scores, int B, int N, int k, int32_
 safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
                            void* O_S, float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
                            void* stream);
+
+/*
+ * SRSU with the global keys assembled in the kernel, Eq. (14), (16): the key
+ * and value rows of S come from the current sensitive rows, all other rows
+ * from the context cache, in original token order; the cache is only read.
+ * The result is bit-identical to safe_ctx_cache_scatter(Kcur, Vcur,
+ * cur_compact, S, ...) into the cache followed by safe_srsu_attn on it, without
+ * the scatter pass and without writing the cache (between anchors its rows of
+ * S are never read as context, Eq. (14), (19)).
+ *  Q          as safe_srsu_attn.
+ *  S          device int32 [B, k], strictly ascending (as safe_topk_partition
+ *             writes it), values in [0, N): it locates the rows of S inside
+ *             each key tile. A row met out of order is skipped and sets bit
+ *             (1 << SAFE_ERR_DEVICE_CHECK) in the device status word.
+ *  Kcur, Vcur device bf16: cur_compact = 1: [B, k, H, d] (row r holds token
+ *             S[b, r]); cur_compact = 0: [B, N, H, d] (rows S[b, r] are used).
+ *  Kc, Vc     device bf16 [B, N, H, d], the context cache (read only).
+ *  O_S, lse, ws, scale: as safe_srsu_attn.
+ */
+safe_status safe_srsu_attn_assembled(const void* Q, int q_compact, const int32_t* S, int k, const void* Kcur,
+                                     const void* Vcur, int cur_compact, const void* Kc, const void* Vc, void* O_S,
+                                     float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
+                                     void* stream);
 
 /*
  * Context-cache update, Eq. (14), (16), (19): write the current sensitive

@@ -12,7 +12,12 @@
 //   warps 1, 2   MMA issuers (one thread each; tile 0 / tile 1): S_t = Q_t K_j^T
 //                into TMEM (SS form), O_t += P_t V_j with P read from TMEM
 //                (TS form). With D = 128 warp 1 issues for both tiles.
-//   warp 3       idle (it completes warpgroup 0)
+//   warp 3       assembled-key SRSU only (kAsm): the key / value tiles come
+//                from the context cache by TMA, and this warp overwrites in
+//                each stage the rows of S with the current rows before the
+//                MMA issuers may read it (Eq. (16): K and V of S u C in token
+//                order, from current sensitive and cached context rows);
+//                otherwise idle (it completes warpgroup 0)
 //   warps 4..7   softmax of tile 0, warps 8..11 softmax of tile 1: one
 //                thread per query row (one TMEM lane); running max / sum in
 //                registers; O rescaled lazily; final O = O_t / l (bf16) and
@@ -98,6 +103,11 @@ struct FlashParams {
   int B, N, H, n_q;
   float scale_log2;       // logit scale * log2(e)
   int gather;
+  // assembled-key mode: the current K / V rows of S, [B, n_q, H, D]
+  // (cur_compact = 1, row r holds token S[b, r]) or [B, N, H, D]
+  const __nv_bfloat16* k_cur;
+  const __nv_bfloat16* v_cur;
+  int cur_compact;
   // Work units are (b, h, 256-row block), ordered with the row block
   // fastest. The first `full_units` CTAs take one whole unit each; the
   // remaining units are split along the key range into `split` parts, one
@@ -117,7 +127,7 @@ constexpr uint32_t kRegsControl = 104, kRegsSoftmax = 200;
 template <int D>
 __host__ __device__ constexpr int flash_smem_bytes() {
   using C = TileCfg<D>;
-  return 1024 /*align slack*/ + (2 + 2 * C::kStages) * C::kTileBytes + 256 /*barriers + tmem slot*/;
+  return 1024 /*align slack*/ + (2 + 2 * C::kStages) * C::kTileBytes + 512 /*barriers + tmem slot*/;
 }
 
 // Combines the key-range parts of the split units: one warp per query row,
@@ -177,7 +187,128 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
+// Byte offset, inside a K stage buffer (K-major chunks, see TileCfg), of the
+// 16-byte unit u (head-dim columns [8u, 8u + 8)) of key row r, with the
+// chunk's swizzle applied as the TMA copy of the tile applies it: the unit
+// index XOR (r mod 8) for 128-byte rows, XOR ((r / 2) mod 4) for 64-byte rows.
 template <int D>
+__device__ __forceinline__ uint32_t k_unit_off(int r, int u) {
+  using C = TileCfg<D>;
+  const int c = u >> 3, uc = u & 7;
+  const int rb = C::row_bytes(c);
+  const int xr = rb == 128 ? (r & 7) : ((r >> 1) & 3);
+  return C::chunk_off(c) + static_cast<uint32_t>(r * rb + ((uc ^ xr) << 4));
+}
+
+// The same for a V stage buffer (equal-width MN-major chunks of kVW columns).
+template <int D>
+__device__ __forceinline__ uint32_t v_unit_off(int r, int u) {
+  using C = TileCfg<D>;
+  constexpr int U = C::kVW / 8;  // units per chunk row
+  const int c = u / U, uc = u % U;
+  const int xr = U == 8 ? (r & 7) : ((r >> 1) & 3);
+  return static_cast<uint32_t>(c) * C::kVChunkBytes + static_cast<uint32_t>(r * C::kVW * 2 + ((uc ^ xr) << 4));
+}
+
+// Assembled-key mode, run by one warp: for each key tile of the CTA, wait for
+// the cache copy of K_j and V_j, overwrite the rows that belong to S with the
+// current rows, and release the stage (k_ready, v_ready). S is ascending, so
+// the rows of S inside tile j are one run of S that starts where the previous
+// tile's run ended (the first run by binary search); each lane copies one row
+// of a 32-row round of the run. A row is checked to lie inside the tile
+// before it is copied (a row out of order is skipped and flagged).
+// Stage j - 1 is released after stage j's copies are issued when K_j / V_j
+// have already landed (its copy latency then overlaps that work), else
+// before waiting for them: a release never waits for a TMA copy, so the
+// stages cannot wait on each other in a cycle, and the prefetch depth of the
+// ring is kept.
+template <int D>
+__device__ void assemble_current_rows(const FlashParams& p, uint8_t* sK, uint8_t* sV, uint64_t* k_full,
+                                      uint64_t* v_full, uint64_t* k_ready, uint64_t* v_ready, int b, int h, int kv0,
+                                      int n_kv, volatile int* abort) {
+  using C = TileCfg<D>;
+  constexpr int ST = C::kStages, TB = C::kTileBytes, UPR = D / 8;
+  const int lane = threadIdx.x & 31;
+  const int32_t* Sb = p.S + static_cast<size_t>(b) * p.n_q;
+  const size_t pitch = static_cast<size_t>(p.H) * D;  // elements from one token row to the next
+  const size_t base = static_cast<size_t>(b) * (p.cur_compact ? p.n_q : p.N) * pitch + static_cast<size_t>(h) * D;
+  const __nv_bfloat16* kb = p.k_cur + base;
+  const __nv_bfloat16* vb = p.v_cur + base;
+  // the copies are generic-proxy writes: each lane waits for its own, fences
+  // them towards the tensor cores' async proxy and then arrives
+  auto release = [&](int stage) {
+    fence_proxy_async_smem();
+    mbar_arrive(&k_ready[stage]);
+    mbar_arrive(&v_ready[stage]);
+  };
+  // first entry of S at or after this CTA's first key
+  int lo = 0, hi = p.n_q;
+  const int first = kv0 * 128;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(Sb + mid) < first)
+      lo = mid + 1;
+    else
+      hi = mid;
+  }
+  int cur = lo;
+  bool bad = false, ok = true;
+  // first round of each tile's run: entry cur + lane of S, loaded ahead
+  int i = cur + lane;
+  int key = i < p.n_q ? __ldg(Sb + i) : INT_MAX;
+  for (int j = 0; j < n_kv; ++j) {
+    const int s = j % ST;
+    const uint32_t par = (j / ST) & 1;
+    const int j0 = (kv0 + j) * 128;
+    const int lim = j0 + 128 < p.N ? j0 + 128 : p.N;
+    bool prev_open = j > 0;  // stage j - 1 not yet released
+    if (prev_open) {
+      const int landed = lane == 0 ? static_cast<int>(mbar_test(&k_full[s], par) && mbar_test(&v_full[s], par)) : 0;
+      if (!__shfl_sync(0xffffffffu, landed, 0)) {
+        cp_async_wait<0>();
+        release((j - 1) % ST);
+        prev_open = false;
+      }
+    }
+    if (!warp_wait(&k_full[s], par, abort) || !warp_wait(&v_full[s], par, abort)) {
+      ok = false;
+      break;
+    }
+    const uint32_t k_dst = smem_u32(sK + s * TB), v_dst = smem_u32(sV + s * TB);
+    for (;;) {
+      const unsigned in = __ballot_sync(0xffffffffu, key < lim);
+      const int run = in == 0xffffffffu ? 32 : __ffs(~in) - 1;  // leading lanes inside the tile
+      if (lane < run) {
+        const int r = key - j0;  // key < lim holds for these lanes
+        if (r < 0) {
+          bad = true;
+        } else {
+          const size_t row = p.cur_compact ? static_cast<size_t>(i) : static_cast<size_t>(key);
+          const __nv_bfloat16* ks = kb + row * pitch;
+          const __nv_bfloat16* vs = vb + row * pitch;
+#pragma unroll
+          for (int u = 0; u < UPR; ++u) cp_async16(k_dst + k_unit_off<D>(r, u), ks + 8 * u);
+#pragma unroll
+          for (int u = 0; u < UPR; ++u) cp_async16(v_dst + v_unit_off<D>(r, u), vs + 8 * u);
+        }
+      }
+      cur += run;
+      i = cur + lane;
+      key = i < p.n_q ? __ldg(Sb + i) : INT_MAX;  // next round, or the next tile's first
+      if (run < 32) break;
+    }
+    cp_async_commit();
+    if (prev_open) {
+      cp_async_wait<1>();  // every group but this stage's
+      release((j - 1) % ST);
+    }
+  }
+  cp_async_wait<0>();
+  if (ok && n_kv > 0) release((n_kv - 1) % ST);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(1 << 5);
+}
+
+template <int D, bool kAsm>
 __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __grid_constant__ FlashParams p) {
   using C = TileCfg<D>;
   constexpr int ST = C::kStages;
@@ -199,7 +330,9 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   uint64_t* pv_done = p_full + 2;    // [2] P_t V complete
   uint64_t* o_full = pv_done + 2;    // [2] last P_t V complete
   uint64_t* drain = o_full + 2;      // [2] per MMA issuer, abort path only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* k_ready = drain + 2;     // [ST] assembled mode: rows of S written into K_j (32 arrivals)
+  uint64_t* v_ready = k_ready + ST;  // [ST] ... and into V_j
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_ready + ST);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -225,6 +358,8 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], kSepP ? 2 : 1);  // one commit per MMA issuer
+      mbar_init(&k_ready[s], 32);  // every lane of the assembling warp
+      mbar_init(&v_ready[s], 32);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -319,6 +454,10 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
         auto tS = [&](int t) -> uint32_t { return tbase + 128u * t; };
         auto tO = [&](int t) -> uint32_t { return tbase + C::kColO + static_cast<uint32_t>(D) * t; };
         auto tP = [&](int t) -> uint32_t { return kSepP ? tbase + C::kColP : tbase + 128u * t; };
+        // stage barriers the MMAs wait on: the TMA copy, or, with assembled
+        // keys, the rows of S written over it
+        uint64_t* k_in = kAsm ? k_ready : k_full;
+        uint64_t* v_in = kAsm ? v_ready : v_full;
         // Descriptors of stage 0 / k-step 0; a k-step or a stage only moves
         // the start address (low 14 bits, in 16-byte units), so each MMA
         // adds a constant to the low word.
@@ -347,7 +486,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
             umma_ts(tO(t), tP(t) + kk * 8, (dV & 0xFFFFFFFF00000000ull) | v, idPV, (j > 0 || kk > 0) ? 1u : 0u);
           }
         };
-        bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&k_full[0], 0, &abort_flag);
+        bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&k_in[0], 0, &abort_flag);
         if (ok) {
           tc_fence_after();
           if constexpr (kSepP) {
@@ -359,14 +498,14 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
               const int s = j % ST;
               if (j + 1 < n_kv) {
                 const int s1 = (j + 1) % ST;
-                ok = mbar_wait(&k_full[s1], ((j + 1) / ST) & 1, &abort_flag) &&
+                ok = mbar_wait(&k_in[s1], ((j + 1) / ST) & 1, &abort_flag) &&
                      mbar_wait(&s_free[mt], j & 1, &abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 issue_S(mt, s1);
                 umma_commit(&s_full[mt]);
               }
-              ok = mbar_wait(&v_full[s], (j / ST) & 1, &abort_flag) && mbar_wait(&p_full[mt], j & 1, &abort_flag);
+              ok = mbar_wait(&v_in[s], (j / ST) & 1, &abort_flag) && mbar_wait(&p_full[mt], j & 1, &abort_flag);
               if (!ok) break;
               tc_fence_after();
               issue_PV(mt, s, j);
@@ -383,7 +522,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
             const int s = j % ST;
             {
               // P overwrites S_t: the next S_t follows P_t V
-              ok = mbar_wait(&v_full[s], (j / ST) & 1, &abort_flag);
+              ok = mbar_wait(&v_in[s], (j / ST) & 1, &abort_flag);
               for (int t = 0; t < 2 && ok; ++t) {
                 ok = mbar_wait(&p_full[t], j & 1, &abort_flag);
                 if (!ok) break;
@@ -392,7 +531,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
                 if (j + 1 < n_kv) {
                   const int s1 = (j + 1) % ST;
                   if (t == 0) {
-                    ok = mbar_wait(&k_full[s1], ((j + 1) / ST) & 1, &abort_flag);
+                    ok = mbar_wait(&k_in[s1], ((j + 1) / ST) & 1, &abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                   }
@@ -413,6 +552,9 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
           mbar_wait_drain(&drain[warp - 1], 0);
         }
       }
+    } else if (kAsm && warp == 3) {
+      // ---------------------------------------------------------- rows of S
+      assemble_current_rows<D>(p, sK, sV, k_full, v_full, k_ready, v_ready, b, h, kv0, n_kv, &abort_flag);
     }
   } else {
     regs_alloc<kRegsSoftmax>();

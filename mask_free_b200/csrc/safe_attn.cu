@@ -22,7 +22,7 @@ using namespace safe;
 
 namespace {
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -164,13 +164,13 @@ FlashPlan plan_flash(int B, int H, int n_q, int N, int d, int sms) {
   return pl;
 }
 
-template <int D>
+template <int D, bool kAsm>
 safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t s) {
   constexpr int smem = flash_smem_bytes<D>();
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(flash_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attr_err = cudaFuncSetAttribute(flash_fwd_kernel<D, kAsm>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   FlashPlan pl = plan_flash(p.B, p.H, p.n_q, p.N, D, device_sms());
@@ -190,16 +190,18 @@ safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t
     p.ws_ml = reinterpret_cast<float2*>(w + pl.ws_ml);
   }
   const unsigned grid = static_cast<unsigned>(pl.full + pl.tail * pl.split);
-  flash_fwd_kernel<D><<<grid, kFlashThreads, smem, s>>>(p);
+  flash_fwd_kernel<D, kAsm><<<grid, kFlashThreads, smem, s>>>(p);
   if (pl.split > 1) flash_merge_kernel<D><<<(pl.tail * 256 + 7) / 8, 256, 0, s>>>(p, pl.tail);
   return launch_status();
 }
 
-safe_status dispatch_flash(int d, FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t s) {
+// assembled: SRSU with the keys of S taken from p.k_cur / p.v_cur
+safe_status dispatch_flash(int d, FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t s, bool assembled = false) {
   switch (d) {
-    case 64: return launch_flash<64>(p, ws, ws_bytes, s);
-    case 96: return launch_flash<96>(p, ws, ws_bytes, s);
-    case 128: return launch_flash<128>(p, ws, ws_bytes, s);
+    case 64: return assembled ? launch_flash<64, true>(p, ws, ws_bytes, s) : launch_flash<64, false>(p, ws, ws_bytes, s);
+    case 96: return assembled ? launch_flash<96, true>(p, ws, ws_bytes, s) : launch_flash<96, false>(p, ws, ws_bytes, s);
+    case 128:
+      return assembled ? launch_flash<128, true>(p, ws, ws_bytes, s) : launch_flash<128, false>(p, ws, ws_bytes, s);
     default: return SAFE_ERR_UNSUPPORTED;
   }
 }
@@ -314,6 +316,29 @@ safe_status noalloc_scratch(void** out) {
   return SAFE_OK;
 }
 
+// Parameters of an SRSU launch (tensor maps of Q or its gather map and of the
+// cache K / V); false when a map cannot be encoded.
+bool fill_srsu(FlashParams& p, const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
+               void* O_S, float* lse, int B, int N, int H, int d, float scale) {
+  if (!encode_v_map(&p.v_map, Vc, B, N, H, d)) return false;
+  for (int c = 0; c < nchunks(d); ++c) {
+    bool ok = encode_rows_map(&p.k_map[c], Kc, B, N, H, d, c);
+    ok = ok && (q_compact ? encode_rows_map(&p.q_map[c], Q, B, k, H, d, c)
+                          : encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c));
+    if (!ok) return false;
+  }
+  p.S = S;
+  p.O = static_cast<__nv_bfloat16*>(O_S);
+  p.lse = lse;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.n_q = k;
+  p.scale_log2 = scale * kLog2e;
+  p.gather = q_compact ? 0 : 1;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -415,23 +440,25 @@ safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k
   if (!q_compact && S == nullptr) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
-  if (!encode_v_map(&p.v_map, Vc, B, N, H, d)) return SAFE_ERR_CUDA;
-  for (int c = 0; c < nchunks(d); ++c) {
-    bool ok = encode_rows_map(&p.k_map[c], Kc, B, N, H, d, c);
-    ok = ok && (q_compact ? encode_rows_map(&p.q_map[c], Q, B, k, H, d, c)
-                          : encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c));
-    if (!ok) return SAFE_ERR_CUDA;
-  }
-  p.S = S;
-  p.O = static_cast<__nv_bfloat16*>(O_S);
-  p.lse = lse;
-  p.B = B;
-  p.N = N;
-  p.H = H;
-  p.n_q = k;
-  p.scale_log2 = scale * kLog2e;
-  p.gather = q_compact ? 0 : 1;
+  if (!fill_srsu(p, Q, q_compact, S, k, Kc, Vc, O_S, lse, B, N, H, d, scale)) return SAFE_ERR_CUDA;
   return dispatch_flash(d, p, ws, ws_bytes, as_stream(stream));
+}
+
+safe_status safe_srsu_attn_assembled(const void* Q, int q_compact, const int32_t* S, int k, const void* Kcur,
+                                     const void* Vcur, int cur_compact, const void* Kc, const void* Vc, void* O_S,
+                                     float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O_S) || !aligned16(Kcur) ||
+      !aligned16(Vcur) || S == nullptr)
+    return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || k < 1 || k > N || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
+  FlashParams p{};
+  if (!fill_srsu(p, Q, q_compact, S, k, Kc, Vc, O_S, lse, B, N, H, d, scale)) return SAFE_ERR_CUDA;
+  p.k_cur = static_cast<const __nv_bfloat16*>(Kcur);
+  p.v_cur = static_cast<const __nv_bfloat16*>(Vcur);
+  p.cur_compact = cur_compact ? 1 : 0;
+  return dispatch_flash(d, p, ws, ws_bytes, as_stream(stream), true);
 }
 
 safe_status safe_attn_cross(const void* Q, const int32_t* q_idx, int nq, const void* Ky, const void* Vy,

@@ -36,6 +36,8 @@ _SIGS = {
     "safe_pcsp_topk": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp],
     "safe_topk_partition": [_vp, _i, _i, _i, _vp, _vp, _vp],
     "safe_srsu_attn": [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp],
+    "safe_srsu_attn_assembled": [_vp, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz,
+                                 _vp],
     "safe_ctx_cache_scatter": [_vp, _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp],
     "safe_get_device_status": [ctypes.POINTER(ctypes.c_int), _vp],
     "safe_status_string": [_i],
@@ -279,6 +281,28 @@ def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=N
     _check("safe_srsu_attn", lib().safe_srsu_attn(_p(Q), 1 if q_compact else 0, _p(S), k, _p(Kc), _p(Vc), _p(out),
                                                   _p(lse if return_lse else None), B, N, H, d, _scale(d, scale),
                                                   _p(w), wb, _stream()))
+    return (out, lse) if return_lse else out
+
+
+def srsu_attn_assembled(Q, S, Kcur, Vcur, Kc, Vc, q_compact=False, cur_compact=False, scale=None, return_lse=False,
+                        out=None, lse=None, ws=None):
+    """SRSU (Eq. (16)) with K/V of S u C assembled in the kernel (Eq. (14)):
+    rows of S from the current Kcur/Vcur ([B, k, H, d] when cur_compact, else
+    [B, N, H, d]), the other rows from the cache Kc/Vc, which is not written.
+    S must be strictly ascending."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(S, "S", torch.int32, 2)
+    for t, n in ((Kcur, "Kcur"), (Vcur, "Vcur"), (Kc, "Kc"), (Vc, "Vc")):
+        _need(t, n, torch.bfloat16, 4)
+    B, N, H, d = Kc.shape
+    k = S.shape[1]
+    out = torch.empty((B, k, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, k), dtype=torch.float32, device=Q.device)
+    w, wb = _attn_ws(ws, B, k, N, H, d, Q.device)
+    _check("safe_srsu_attn_assembled", lib().safe_srsu_attn_assembled(
+        _p(Q), 1 if q_compact else 0, _p(S), k, _p(Kcur), _p(Vcur), 1 if cur_compact else 0, _p(Kc), _p(Vc), _p(out),
+        _p(lse if return_lse else None), B, N, H, d, _scale(d, scale), _p(w), wb, _stream()))
     return (out, lse) if return_lse else out
 
 

@@ -47,7 +47,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.safe_abi_version() == 3
+    assert lib.safe_abi_version() == 4
     assert lib.safe_status_string(0) == b"ok"
     assert lib.safe_status_string(1) == b"invalid argument"
     assert lib.safe_status_string(99) == b"unknown status"
@@ -82,6 +82,14 @@ def test_host_validation_rejects_bad_arguments_without_gpu(lib):
     # SRSU: k out of range
     assert lib.safe_srsu_attn(fake, 0, fake, 0, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
     assert lib.safe_srsu_attn(fake, 0, fake, 17, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    # assembled-key SRSU: S and the current rows are required; k, d as above
+    asm = lib.safe_srsu_attn_assembled
+    assert asm(fake, 0, null, 4, fake, fake, 1, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert asm(fake, 0, fake, 4, null, fake, 1, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert asm(fake, 0, fake, 4, fake, odd, 1, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert asm(fake, 0, fake, 0, fake, fake, 1, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert asm(fake, 0, fake, 17, fake, fake, 1, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
+    assert asm(fake, 0, fake, 4, fake, fake, 1, fake, fake, fake, null, 1, 16, 1, 80, 1.0, null, 0, null) == 2
     # cross: M > 256 unsupported, nq must equal N without q_idx
     assert lib.safe_attn_cross(fake, null, 16, fake, fake, fake, fake, 1, 16, 257, 1, 96, 1.0, null) == 2
     assert lib.safe_attn_cross(fake, null, 8, fake, fake, fake, fake, 1, 16, 16, 1, 96, 1.0, null) == 1
@@ -162,4 +170,4 @@ def test_graft_entry_build_loads_the_library():
     # checks the ABI version it was written against
     import __graft_entry__ as g
     g.build()
-    assert ops.abi_version() == 3
+    assert ops.abi_version() == 4
