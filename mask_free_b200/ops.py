@@ -99,15 +99,55 @@ def _p(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _need(t: torch.Tensor, name: str, dtype, ndim: int):
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+def _on_device(t: torch.Tensor) -> bool:
+    return t.is_cuda
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int, shape=None, device=None):
+    """Check a tensor argument: a contiguous CUDA tensor of `dtype` and `ndim`
+    dims; with `shape` exactly that shape, with `device` on that device. The
+    library trusts the sizes it is given, so every tensor whose extent follows
+    from another argument is checked here before any launch."""
+    if not isinstance(t, torch.Tensor) or not _on_device(t):
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _out(t, name: str, dtype, shape, device):
+    """An output buffer: a new one, or the given one checked like an input."""
+    if t is None:
+        return torch.empty(tuple(shape), dtype=dtype, device=device)
+    _need(t, name, dtype, len(shape), shape, device)
+    return t
+
+
+def _text_kv(Ky, Vy, B, H, d, device):
+    """Check the text keys / values [B, M, H, d]; returns M."""
+    _need(Ky, "Ky", torch.bfloat16, 4, device=device)
+    M = Ky.shape[1]
+    _need(Ky, "Ky", torch.bfloat16, 4, (B, M, H, d), device)
+    if Vy is not None:
+        _need(Vy, "Vy", torch.bfloat16, 4, (B, M, H, d), device)
+    return M
+
+
+def _split_bufs(S, C, B, N, k, device, with_c=True):
+    """S [B, k] and C [B, N - k] int32 buffers of the top-k split."""
+    if k > N:
+        raise ValueError(f"k = {k} exceeds N = {N}")
+    S = _out(S, "S", torch.int32, (B, k), device)
+    if with_c:
+        C = _out(C, "C", torch.int32, (B, N - k), device)
+    return S, C
 
 
 def abi_version() -> int:
@@ -118,12 +158,11 @@ def mask_classify(mask: torch.Tensor, sync: bool = True, result: Optional[torch.
     """Row-constant mask classification (Eq. (6)) of a 4-D [B, H, n_q, n_k]
     mask view (any strides; stride 0 = broadcast). Returns (verdict, nfail,
     first_fail) as Python ints when sync, else the device int64[3] tensor."""
-    if mask.dim() != 4 or not mask.is_cuda or mask.dtype not in _MASK_DTYPES:
+    if not isinstance(mask, torch.Tensor) or mask.dim() != 4 or not _on_device(mask) or mask.dtype not in _MASK_DTYPES:
         raise ValueError("mask must be a 4-D CUDA tensor of dtype bool/uint8/float32/float16/bfloat16")
     sizes = (ctypes.c_int64 * 4)(*mask.shape)
     strides = (ctypes.c_int64 * 4)(*mask.stride())
-    if result is None:
-        result = torch.empty(3, dtype=torch.int64, device=mask.device)
+    result = _out(result, "result", torch.int64, (3,), mask.device)
     if sync:
         h = (ctypes.c_int64 * 3)()
         _check("safe_mask_classify_sync",
@@ -158,14 +197,14 @@ def _attn_ws(ws, B, n_q, N, H, d, device):
 
 def attn_self(Q, K, V, scale=None, return_lse=False, out=None, lse=None, ws=None):
     """Mask-free image self-attention (Eq. (3) with the mask elided)."""
-    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
-        _need(t, n, torch.bfloat16, 4)
+    _need(Q, "Q", torch.bfloat16, 4)
     B, N, H, d = Q.shape
-    if K.shape != Q.shape or V.shape != Q.shape:
-        raise ValueError("Q, K, V must share the shape [B, N, H, d]")
-    out = torch.empty_like(Q) if out is None else out
-    if return_lse and lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    dev = Q.device
+    _need(K, "K", torch.bfloat16, 4, Q.shape, dev)
+    _need(V, "V", torch.bfloat16, 4, Q.shape, dev)
+    out = _out(out, "out", torch.bfloat16, (B, N, H, d), dev)
+    if return_lse:
+        lse = _out(lse, "lse", torch.float32, (B, H, N), dev)
     w, wb = _attn_ws(ws, B, N, N, H, d, Q.device)
     _check("safe_attn_self", lib().safe_attn_self(_p(Q), _p(K), _p(V), _p(out), _p(lse if return_lse else None),
                                                   B, N, H, d, _scale(d, scale), _p(w), wb, _stream()))
@@ -176,16 +215,16 @@ def attn_cross(Q, Ky, Vy, valid_len, q_idx=None, scale=None, out=None):
     """Image->text cross-attention with the padding kept as valid lengths
     (Eq. (4)); with q_idx = S the row-selective form (Eq. (17))."""
     _need(Q, "Q", torch.bfloat16, 4)
-    _need(Ky, "Ky", torch.bfloat16, 4)
-    _need(Vy, "Vy", torch.bfloat16, 4)
-    _need(valid_len, "valid_len", torch.int32, 1)
     B, N, H, d = Q.shape
-    M = Ky.shape[1]
+    dev = Q.device
+    M = _text_kv(Ky, Vy, B, H, d, dev)
+    _need(valid_len, "valid_len", torch.int32, 1, (B,), dev)
     nq = N
     if q_idx is not None:
-        _need(q_idx, "q_idx", torch.int32, 2)
+        _need(q_idx, "q_idx", torch.int32, 2, device=dev)
         nq = q_idx.shape[1]
-    out = torch.empty((B, nq, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
+        _need(q_idx, "q_idx", torch.int32, 2, (B, nq), dev)
+    out = _out(out, "out", torch.bfloat16, (B, nq, H, d), dev)
     _check("safe_attn_cross", lib().safe_attn_cross(_p(Q), _p(q_idx), nq, _p(Ky), _p(Vy), _p(valid_len), _p(out),
                                                     B, N, M, H, d, _scale(d, scale), _stream()))
     return out
@@ -200,23 +239,23 @@ def pcsp_topk(Q, Ky, valid_len, w=None, scores=None, accumulate=False, k=0, scal
     partition (Eq. (12)). Returns (scores, S, C)."""
     if Q is not None:
         _need(Q, "Q", torch.bfloat16, 4)
-        _need(Ky, "Ky", torch.bfloat16, 4)
-        _need(valid_len, "valid_len", torch.int32, 1)
         B, N, H, d = Q.shape
-        M = Ky.shape[1]
         dev = Q.device
+        M = _text_kv(Ky, None, B, H, d, dev)
+        _need(valid_len, "valid_len", torch.int32, 1, (B,), dev)
+        if w is not None:
+            _need(w, "w", torch.float32, 2, (B, M), dev)
     else:
         _need(scores, "scores", torch.float32, 2)
         B, N = scores.shape
         H, d, M = 1, 64, 1
         dev = scores.device
-    if w is not None:
-        _need(w, "w", torch.float32, 2)
     if scores is None:
         scores = torch.zeros((B, N), dtype=torch.float32, device=dev)
+    else:
+        _need(scores, "scores", torch.float32, 2, (B, N), dev)
     if k > 0:
-        S = torch.empty((B, k), dtype=torch.int32, device=dev) if S is None else S
-        C = torch.empty((B, N - k), dtype=torch.int32, device=dev) if C is None else C
+        S, C = _split_bufs(S, C, B, N, k, dev)
     nbytes = pcsp_workspace_bytes(B, N, H) if Q is not None else 0
     if Q is not None and ws is None:
         ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
@@ -232,19 +271,19 @@ def attn_cross_pcsp(Q, Ky, Vy, valid_len, w=None, out=None, scores=None, accumul
     probabilities, in one pass over Q; with k > 0 also the top-k split
     (Eq. (12)). Returns (O, scores, S, C)."""
     _need(Q, "Q", torch.bfloat16, 4)
-    _need(Ky, "Ky", torch.bfloat16, 4)
-    _need(Vy, "Vy", torch.bfloat16, 4)
-    _need(valid_len, "valid_len", torch.int32, 1)
-    if w is not None:
-        _need(w, "w", torch.float32, 2)
     B, N, H, d = Q.shape
-    M = Ky.shape[1]
-    out = torch.empty_like(Q) if out is None else out
+    dev = Q.device
+    M = _text_kv(Ky, Vy, B, H, d, dev)
+    _need(valid_len, "valid_len", torch.int32, 1, (B,), dev)
+    if w is not None:
+        _need(w, "w", torch.float32, 2, (B, M), dev)
+    out = _out(out, "out", torch.bfloat16, (B, N, H, d), dev)
     if scores is None:
-        scores = torch.zeros((B, N), dtype=torch.float32, device=Q.device)
+        scores = torch.zeros((B, N), dtype=torch.float32, device=dev)
+    else:
+        _need(scores, "scores", torch.float32, 2, (B, N), dev)
     if k > 0:
-        S = torch.empty((B, k), dtype=torch.int32, device=Q.device) if S is None else S
-        C = torch.empty((B, N - k), dtype=torch.int32, device=Q.device) if C is None else C
+        S, C = _split_bufs(S, C, B, N, k, dev)
     if ws is None:
         ws = torch.empty(max(pcsp_workspace_bytes(B, N, H), 256), dtype=torch.uint8, device=Q.device)
     _check("safe_attn_cross_pcsp", lib().safe_attn_cross_pcsp(
@@ -257,27 +296,34 @@ def topk_partition(scores, k, S=None, C=None, with_c=True):
     """Exact tie-stable top-k split of Eq. (12) on given scores."""
     _need(scores, "scores", torch.float32, 2)
     B, N = scores.shape
-    S = torch.empty((B, k), dtype=torch.int32, device=scores.device) if S is None else S
-    if with_c and C is None:
-        C = torch.empty((B, N - k), dtype=torch.int32, device=scores.device)
+    S, C = _split_bufs(S, C, B, N, k, scores.device, with_c)
     _check("safe_topk_partition", lib().safe_topk_partition(_p(scores), B, N, k, _p(S), _p(C if with_c else None),
                                                             _stream()))
     return S, C
 
 
+def _srsu_args(Q, S, Kc, Vc, q_compact):
+    """Check the SRSU inputs: cache K/V [B, N, H, d], S [B, k], Q [B, k, H, d]
+    (compact) or [B, N, H, d]; returns B, N, H, d, k, device."""
+    _need(Kc, "Kc", torch.bfloat16, 4)
+    B, N, H, d = Kc.shape
+    dev = Kc.device
+    _need(Vc, "Vc", torch.bfloat16, 4, Kc.shape, dev)
+    _need(S, "S", torch.int32, 2, device=dev)
+    k = S.shape[1]
+    _need(S, "S", torch.int32, 2, (B, k), dev)
+    _need(Q, "Q", torch.bfloat16, 4, (B, k if q_compact else N, H, d), dev)
+    return B, N, H, d, k, dev
+
+
 def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=None, lse=None, ws=None):
     """SRSU selective self-attention (Eq. (16)): rows S of Q against all N
     keys of the assembled global K/V."""
-    _need(Q, "Q", torch.bfloat16, 4)
-    _need(S, "S", torch.int32, 2)
-    _need(Kc, "Kc", torch.bfloat16, 4)
-    _need(Vc, "Vc", torch.bfloat16, 4)
-    B, N, H, d = Kc.shape
-    k = S.shape[1]
-    out = torch.empty((B, k, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
-    if return_lse and lse is None:
-        lse = torch.empty((B, H, k), dtype=torch.float32, device=Q.device)
-    w, wb = _attn_ws(ws, B, k, N, H, d, Q.device)
+    B, N, H, d, k, dev = _srsu_args(Q, S, Kc, Vc, q_compact)
+    out = _out(out, "out", torch.bfloat16, (B, k, H, d), dev)
+    if return_lse:
+        lse = _out(lse, "lse", torch.float32, (B, H, k), dev)
+    w, wb = _attn_ws(ws, B, k, N, H, d, dev)
     _check("safe_srsu_attn", lib().safe_srsu_attn(_p(Q), 1 if q_compact else 0, _p(S), k, _p(Kc), _p(Vc), _p(out),
                                                   _p(lse if return_lse else None), B, N, H, d, _scale(d, scale),
                                                   _p(w), wb, _stream()))
@@ -290,16 +336,14 @@ def srsu_attn_assembled(Q, S, Kcur, Vcur, Kc, Vc, q_compact=False, cur_compact=F
     rows of S from the current Kcur/Vcur ([B, k, H, d] when cur_compact, else
     [B, N, H, d]), the other rows from the cache Kc/Vc, which is not written.
     S must be strictly ascending."""
-    _need(Q, "Q", torch.bfloat16, 4)
-    _need(S, "S", torch.int32, 2)
-    for t, n in ((Kcur, "Kcur"), (Vcur, "Vcur"), (Kc, "Kc"), (Vc, "Vc")):
-        _need(t, n, torch.bfloat16, 4)
-    B, N, H, d = Kc.shape
-    k = S.shape[1]
-    out = torch.empty((B, k, H, d), dtype=torch.bfloat16, device=Q.device) if out is None else out
-    if return_lse and lse is None:
-        lse = torch.empty((B, H, k), dtype=torch.float32, device=Q.device)
-    w, wb = _attn_ws(ws, B, k, N, H, d, Q.device)
+    B, N, H, d, k, dev = _srsu_args(Q, S, Kc, Vc, q_compact)
+    cur_shape = (B, k if cur_compact else N, H, d)
+    _need(Kcur, "Kcur", torch.bfloat16, 4, cur_shape, dev)
+    _need(Vcur, "Vcur", torch.bfloat16, 4, cur_shape, dev)
+    out = _out(out, "out", torch.bfloat16, (B, k, H, d), dev)
+    if return_lse:
+        lse = _out(lse, "lse", torch.float32, (B, H, k), dev)
+    w, wb = _attn_ws(ws, B, k, N, H, d, dev)
     _check("safe_srsu_attn_assembled", lib().safe_srsu_attn_assembled(
         _p(Q), 1 if q_compact else 0, _p(S), k, _p(Kcur), _p(Vcur), 1 if cur_compact else 0, _p(Kc), _p(Vc), _p(out),
         _p(lse if return_lse else None), B, N, H, d, _scale(d, scale), _p(w), wb, _stream()))
@@ -309,13 +353,18 @@ def srsu_attn_assembled(Q, S, Kcur, Vcur, Kc, Vc, q_compact=False, cur_compact=F
 def ctx_cache_scatter(Ksrc, Vsrc, S, Kc, Vc, src_compact=True):
     """In-place cache update (Eq. (14)/(16)); S=None is the anchor refresh
     (Eq. (19))."""
-    for t, n in ((Ksrc, "Ksrc"), (Vsrc, "Vsrc"), (Kc, "Kc"), (Vc, "Vc")):
-        _need(t, n, torch.bfloat16, 4)
+    _need(Kc, "Kc", torch.bfloat16, 4)
     B, N, H, d = Kc.shape
+    dev = Kc.device
+    _need(Vc, "Vc", torch.bfloat16, 4, Kc.shape, dev)
     k = 0
     if S is not None:
-        _need(S, "S", torch.int32, 2)
+        _need(S, "S", torch.int32, 2, device=dev)
         k = S.shape[1]
+        _need(S, "S", torch.int32, 2, (B, k), dev)
+    src_shape = (B, k, H, d) if (src_compact and S is not None) else (B, N, H, d)
+    _need(Ksrc, "Ksrc", torch.bfloat16, 4, src_shape, dev)
+    _need(Vsrc, "Vsrc", torch.bfloat16, 4, src_shape, dev)
     _check("safe_ctx_cache_scatter", lib().safe_ctx_cache_scatter(
         _p(Ksrc), _p(Vsrc), 1 if (src_compact and S is not None) else 0, _p(S), k, _p(Kc), _p(Vc), B, N, H, d,
         _stream()))
@@ -354,7 +403,9 @@ def sensitivity_field(scores, grid_h: int, grid_w: int, sigma: float, truncate: 
     (row-major tokens), per sample: [B, N] fp32 -> [B, N] fp32 in [0, 1]."""
     _need(scores, "scores", torch.float32, 2)
     B, N = scores.shape
-    out = torch.empty_like(scores) if out is None else out
+    if N != grid_h * grid_w:
+        raise ValueError(f"scores hold {N} tokens per sample, the grid {grid_h} x {grid_w} has {grid_h * grid_w}")
+    out = _out(out, "out", torch.float32, (B, N), scores.device)
     nbytes = sensitivity_workspace_bytes(B, N)
     if ws is None:
         ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=scores.device)
@@ -367,7 +418,7 @@ def partition_indicator(S, N: int, out=None):
     """Binary field of the SW-CFG binary variant: 1 on S, 0 on C ([B, N] fp32)."""
     _need(S, "S", torch.int32, 2)
     B, k = S.shape
-    out = torch.empty((B, N), dtype=torch.float32, device=S.device) if out is None else out
+    out = _out(out, "out", torch.float32, (B, N), S.device)
     _check("safe_partition_indicator", lib().safe_partition_indicator(_p(S), k, _p(out), B, N, _stream()))
     return out
 
@@ -382,10 +433,11 @@ def sw_cfg(f_c, f_u, s, gamma_ctx: float, gamma_sens: float, out=None):
     if f_c.dtype not in _CFG_DTYPES or f_u.dtype != f_c.dtype:
         raise ValueError("f_c and f_u must both be float32 or both bfloat16")
     _need(f_c, "f_c", f_c.dtype, 3)
-    _need(f_u, "f_u", f_c.dtype, 3)
-    _need(s, "s", torch.float32, 2)
     B, N, C = f_c.shape
-    out = torch.empty_like(f_c) if out is None else out
+    dev = f_c.device
+    _need(f_u, "f_u", f_c.dtype, 3, f_c.shape, dev)
+    _need(s, "s", torch.float32, 2, (B, N), dev)
+    out = _out(out, "out", f_c.dtype, (B, N, C), dev)
     _check("safe_sw_cfg", lib().safe_sw_cfg(_p(f_c), _p(f_u), _p(s), _p(out), _CFG_DTYPES[f_c.dtype], B, N, C,
                                             float(gamma_ctx), float(gamma_sens), _stream()))
     return out
