@@ -10,4 +10,5 @@ from .safe_oracle import (DTYPE_BF16, DTYPE_BOOL, DTYPE_F16, DTYPE_F32, DTYPE_U8
                           attention, cache_scatter, ceil_k, classify_mask, cross_attention,
                           pcsp_scores, row_in_R, sdpa_masked, softmax_rows, srsu_attention,
                           text_probabilities, topk_partition, gaussian_taps, reflect_index, smooth_scores,
-                          norm01, sensitivity_field, partition_indicator, sw_cfg)
+                          norm01, sensitivity_field, partition_indicator, sw_cfg, gelu_tanh,
+                          gathered_linear)

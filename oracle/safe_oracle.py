@@ -413,3 +413,44 @@ def sw_cfg(f_c: np.ndarray, f_u: np.ndarray, s: np.ndarray, gamma_ctx: float,
     fu = np.asarray(f_u, dtype=np.float64)
     gamma = gamma_ctx + (gamma_sens - gamma_ctx) * np.asarray(s, dtype=np.float64)
     return fu + gamma[:, :, None] * (fc - fu)
+
+
+# ----------------------------------------------------------------------------
+# Row-selective block: row-wise layers on the rows of S  (Eq. (13), (15))
+# ----------------------------------------------------------------------------
+
+
+def gelu_tanh(x: np.ndarray) -> np.ndarray:
+    """GELU in its tanh form (Hendrycks and Gimpel, "Gaussian Error Linear
+    Units (GELUs)", the tanh approximation of x * Phi(x)):
+        0.5 x (1 + tanh( sqrt(2 / pi) (x + 0.044715 x^3) )).
+    The paper names no activation; this is the form DiT-family MLPs use."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def gathered_linear(X: np.ndarray, S: Optional[np.ndarray], Wt: np.ndarray,
+                    bias: Optional[np.ndarray] = None, act: str = "none") -> np.ndarray:
+    """A row-wise layer of the row-selective block B^S (Eq. (15)) evaluated
+    only on the sensitive rows: with the row selection P_S of Eq. (13),
+
+        Y[b, r, :] = act( X[b, S[b, r], :] @ Wt^T + bias ),
+
+    X [B, N, D_in] (token-major), Wt [D_out, D_in] (the weight of a linear
+    layer y = x W^T + b), bias [D_out] or None, act "none" or "gelu_tanh".
+    S = None selects every row in order (the dense block of Eq. (18)). One
+    library matmul per sample, fp64. Returns [B, k or N, D_out]."""
+    X = np.asarray(X, dtype=np.float64)
+    Wt = np.asarray(Wt, dtype=np.float64)
+    out = []
+    for b in range(X.shape[0]):
+        rows = X[b] if S is None else X[b, np.asarray(S)[b]]   # P_S H (Eq. (13))
+        y = rows @ Wt.T
+        if bias is not None:
+            y = y + np.asarray(bias, dtype=np.float64)[None, :]
+        if act == "gelu_tanh":
+            y = gelu_tanh(y)
+        elif act != "none":
+            raise ValueError(f"unknown activation {act!r}")
+        out.append(y)
+    return np.stack(out)

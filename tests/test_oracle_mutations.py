@@ -113,9 +113,30 @@ def _indicator_complement(S, N):
     return 1.0 - _ORIG["partition_indicator"](S, N)
 
 
+def _linear_transposed_weight(X, Sidx, Wt, bias=None, act="none"):
+    return _ORIG["gathered_linear"](X, Sidx, np.asarray(Wt).T, bias, act)
+
+
+def _linear_bias_after_activation(X, Sidx, Wt, bias=None, act="none"):
+    y = _ORIG["gathered_linear"](X, Sidx, Wt, None, act)
+    return y if bias is None else y + np.asarray(bias)[None, None, :]
+
+
+def _linear_ignores_rows(X, Sidx, Wt, bias=None, act="none"):
+    if Sidx is None:
+        return _ORIG["gathered_linear"](X, None, Wt, bias, act)
+    k = np.asarray(Sidx).shape[1]
+    return _ORIG["gathered_linear"](np.asarray(X)[:, :k], None, Wt, bias, act)
+
+
+def _gelu_cubic_coefficient_slip(x):
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.44715 * x ** 3)))
+
+
 _ORIG = {n: getattr(S, n) for n in ("attention", "softmax_rows", "ceil_k", "topk_partition", "row_in_R",
                                     "pcsp_scores", "cache_scatter", "gaussian_taps", "smooth_scores", "sw_cfg",
-                                    "partition_indicator")}
+                                    "partition_indicator", "gathered_linear")}
 
 MUTATIONS = {
     "attention_no_scale": ("attention", _attention_no_scale),
@@ -134,6 +155,10 @@ MUTATIONS = {
     "sw_cfg_swapped_predictions": ("sw_cfg", _sw_cfg_swapped),
     "sw_cfg_swapped_scales": ("sw_cfg", _sw_cfg_scales_swapped),
     "indicator_complement": ("partition_indicator", _indicator_complement),
+    "linear_transposed_weight": ("gathered_linear", _linear_transposed_weight),
+    "linear_bias_after_activation": ("gathered_linear", _linear_bias_after_activation),
+    "linear_ignores_selected_rows": ("gathered_linear", _linear_ignores_rows),
+    "gelu_cubic_coefficient_slip": ("gelu_tanh", _gelu_cubic_coefficient_slip),
 }
 
 

@@ -507,3 +507,61 @@ def test_partition_indicator_binary_variant():
     for b in range(2):
         for i in range(6):
             np.testing.assert_allclose(out[b, i], fu[b, i] if i in S[b] else fc[b, i], atol=1e-15)
+
+
+# ---------------------------------------------------------------- row-selective block (Eq. (13), (15))
+
+
+def test_gathered_linear_hand_computed():
+    # X rows [1, 2], [3, 4], [5, 6]; W^T maps (a, b) to (a, b, a + b); bias
+    # (0.5, 0, -1). Rows S = (2, 0): (5, 6) -> (5.5, 6, 10), (1, 2) -> (1.5, 2, 2)
+    X = np.array([[[1.0, 2.0], [3.0, 4.0], [5.0, 6.0]]])
+    Wt = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]])
+    got = O.gathered_linear(X, np.array([[2, 0]]), Wt, np.array([0.5, 0.0, -1.0]))
+    assert np.array_equal(got, np.array([[[5.5, 6.0, 10.0], [1.5, 2.0, 2.0]]]))
+    # without S: every row, in order
+    assert np.array_equal(O.gathered_linear(X, None, Wt)[0, 1], np.array([3.0, 4.0, 7.0]))
+
+
+def test_gathered_linear_brute_force_with_activation():
+    import torch
+    rng = np.random.default_rng(3)
+    B, N, Din, Dout = 2, 7, 5, 3
+    X = rng.standard_normal((B, N, Din))
+    Wt = rng.standard_normal((Dout, Din))
+    bias = rng.standard_normal(Dout)
+    S = np.array([[6, 1, 3], [0, 2, 5]])
+    got = O.gathered_linear(X, S, Wt, bias, act="gelu_tanh")
+    for b, r, n in itertools.product(range(B), range(S.shape[1]), range(Dout)):
+        acc = bias[n]
+        for c in range(Din):
+            acc += X[b, S[b, r], c] * Wt[n, c]
+        want = torch.nn.functional.gelu(torch.tensor(acc, dtype=torch.float64), approximate="tanh").item()
+        assert abs(got[b, r, n] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_gathered_linear_row_selection_commutes():
+    # P_S (X W^T) = (P_S X) W^T: the selected rows of the dense layer
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((2, 40, 16))
+    Wt = rng.standard_normal((24, 16))
+    S = np.stack([np.sort(rng.choice(40, 11, replace=False)) for _ in range(2)])
+    dense = O.gathered_linear(X, None, Wt, act="gelu_tanh")
+    sel = O.gathered_linear(X, S, Wt, act="gelu_tanh")
+    for b in range(2):
+        assert np.allclose(sel[b], dense[b, S[b]], rtol=0, atol=1e-12)
+
+
+def test_gelu_tanh_library_odd_part_and_exact_gelu():
+    import torch
+    x = np.linspace(-8.0, 8.0, 3201)
+    g = O.gelu_tanh(x)
+    lib = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    assert np.max(np.abs(g - lib)) <= 1e-12
+    # odd part: gelu(x) - gelu(-x) = x for x * s(x) with s(x) + s(-x) = 1
+    assert np.max(np.abs((g - O.gelu_tanh(-x)) - x)) <= 1e-12
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+    # within 1e-3 of the exact x * Phi(x) everywhere (the approximation's
+    # deviation is a few 1e-4 at most)
+    exact = np.array([0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))) for v in x])
+    assert np.max(np.abs(g - exact)) <= 1e-3
