@@ -319,6 +319,30 @@ def kernel_table(dev, pk):
             out[f"srsu_assembled_{tag}_k{k}"] = {
                 "ms": t_a, "tflops": srsu_f / t_a / 1e9, "pct_bf16_burst": 100 * srsu_f / t_a / 1e9 / pk["bf16"],
                 "scatter_plus_srsu_ms": t_sc + t_s, "saved_ms": t_sc + t_s - t_a}
+            # row-wise layers of the row-selective block (Eq. (15)) at width
+            # H*d = 2304: QKV projection and MLP up (GELU) on the rows of S,
+            # MLP down on the compact hidden rows; context: torch's linear
+            # (cuBLAS) on the same rows already gathered
+            dm = s.H * s.d
+            Xh = torch.randn((s.B, s.N, dm), device=dev).to(torch.bfloat16)
+            lin = {}
+            for name, din, dout, act, rows in (("qkv", dm, 3 * dm, "none", S), ("mlp_up", dm, 4 * dm, "gelu_tanh", S),
+                                               ("mlp_down", 4 * dm, dm, "none", None)):
+                Wl = (torch.randn((dout, din), device=dev) / math.sqrt(din)).to(torch.bfloat16)
+                bl = torch.zeros(dout, device=dev)
+                Xin = Xh if rows is not None else torch.randn((s.B, k, din), device=dev).to(torch.bfloat16)
+                Yl = torch.empty((s.B, k, dout), dtype=torch.bfloat16, device=dev)
+                t_l = time_kernel(lambda: ops.gather_linear(Xin, Wl, S=rows, bias=bl, act=act, out=Yl))
+                fl = 2.0 * s.B * k * din * dout
+                Xg = Xin if rows is None else torch.stack([Xin[b, rows[b].long()] for b in range(s.B)])
+                blh = bl.to(torch.bfloat16)
+                t_cb = time_kernel(lambda: torch.nn.functional.linear(Xg, Wl, blh), reps=10)
+                lin[name] = {"ms": t_l, "tflops": fl / t_l / 1e9, "pct_bf16_burst": 100 * fl / t_l / 1e9 / pk["bf16"],
+                             "d_in": din, "d_out": dout, "act": act, "rows_gathered": rows is not None,
+                             "torch_linear_on_gathered_rows_ms": t_cb}
+                del Wl, Xin, Yl, Xg, blh
+            del Xh
+            out[f"block_linear_{tag}_k{k}"] = lin
             sc = torch.empty((s.B, s.N), dtype=torch.float32, device=dev)
             ws = torch.empty(ops.pcsp_workspace_bytes(s.B, s.N, s.H), dtype=torch.uint8, device=dev)
             t_p = time_kernel(lambda: ops.pcsp_topk(inp["Q"], inp["Ky"], inp["valid_len"], inp["w"], scores=sc, ws=ws))

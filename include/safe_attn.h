@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { SAFE_BOOL = 0, SAFE_U8 = 1, SAFE_F32 = 2, SAFE_F16 = 3, SAFE_BF16 = 4 } safe_dtype;
 
-/* ABI version of this header (bumped on any signature or entry-point change): 4. */
+/* ABI version of this header (bumped on any signature or entry-point change): 5. */
 int safe_abi_version(void);
 const char* safe_status_string(int status);
 
@@ -298,6 +298,26 @@ safe_status safe_partition_indicator(const int32_t* S, int k, float* s, int B, i
  */
 safe_status safe_sw_cfg(const void* f_c, const void* f_u, const float* s, void* out, int dtype, int B, int N, int C,
                         float gamma_ctx, float gamma_sens, void* stream);
+
+/*
+ * A row-wise layer of the row-selective block B^S (Eq. (15)) on the
+ * sensitive rows only; with the row selection P_S of Eq. (13):
+ *   Y[b, r, :] = act( X[b, S[b, r], :] W^T + bias ),   r < k
+ * S == NULL: every row in order (r < N; the dense block of Eq. (18)), k
+ * ignored. bf16 operands, fp32 accumulation on the tensor cores, bf16 result.
+ * The projections and the MLP of the block are such layers; the paper names
+ * no activation: act 0 = none, 1 = GELU in its tanh form
+ * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+ *  X     device bf16 [B, N, d_in], token-major.
+ *  S     device int32 [B, k] rows of X (any order; an index outside [0, N) is
+ *        replaced by row 0 and flagged), or NULL.
+ *  Wt    device bf16 [d_out, d_in] (the weight of y = x W^T + b).
+ *  bias  device fp32 [d_out] (4-byte aligned) or NULL.
+ *  Y     device bf16 [B, k or N, d_out] (written; may not overlap X or Wt).
+ *  d_in >= 64 and d_out >= 8, both multiples of 8; X, Wt, Y 16-byte aligned.
+ */
+safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const void* Wt, const float* bias, int act,
+                               void* Y, int B, int N, int d_in, int d_out, void* stream);
 
 /*
  * Device status word: synchronises `stream`, writes to *h_status (host) the

@@ -1,0 +1,239 @@
+// linear.cuh - row-wise layers of the row-selective block on tcgen05 tensor cores.
+//
+// The row-selective block B^S of SAFE-DiT (Eq. (15)) evaluates its
+// projections and MLP only on the sensitive rows; with the row selection P_S
+// of Eq. (13) each such layer is
+//     Y[b, r, :] = act( X[b, S[b, r], :] W^T + bias )
+// (no S: every row in order, the dense block of Eq. (18)).
+//
+// Persistent kernel: one CTA per SM walks the 128 x 256 output tiles
+// t = blockIdx.x, blockIdx.x + gridDim.x, ... (the column tile fastest, so
+// CTAs running at the same time share their gathered rows of X through L2).
+//   warp 0     producer: per 64-wide K chunk, the 128 rows of X by TMA
+//              gather4 (lane l copies rows 4l .. 4l + 3) and the 256 x 64
+//              tile of W by one tiled copy, both K-major with the 128B
+//              swizzle, into a 4-stage ring
+//   warp 1     MMA issuer: tcgen05.mma M = 128, N = 256, K = 16 into one of
+//              two 256-column TMEM accumulators (tile i uses buffer i & 1)
+//   warp 2     TMEM allocation
+//   warps 4..7 epilogue: tcgen05.ld of the accumulator (TMEM lane = row of
+//              the tile), + bias, activation, bf16 rows to global memory;
+//              the buffer is released once read, so the next tile's MMAs
+//              overlap this tile's stores
+// Every wait is bounded (sm100.cuh); a row index outside [0, N) is flagged
+// and replaced by row 0.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace safe {
+
+struct LinearParams {
+  CUtensorMap x_map;    // 2-D [B*N, d_in], box 64 x 1 (gather4)
+  CUtensorMap w_map;    // 2-D [d_out, d_in], box 64 x 256
+  const int32_t* S;     // [B, R] rows of X, or null (rows 0 .. R-1)
+  const float* bias;    // [d_out] or null
+  __nv_bfloat16* Y;     // [B, R, d_out]
+  int B, N, R, d_in, d_out, act;
+  int m_tiles;          // row tiles per sample: ceil(R / 128)
+  int n_tiles;          // column tiles: ceil(d_out / 256)
+  int tiles;            // B * m_tiles * n_tiles
+};
+
+constexpr int kLinThreads = 256;
+constexpr int kLinStages = 4;
+constexpr int kLinABytes = 128 * 128;  // 128 rows x 64 bf16
+constexpr int kLinBBytes = 256 * 128;  // 256 rows x 64 bf16
+constexpr int kLinSmem = 1024 + kLinStages * (kLinABytes + kLinBBytes) + 256;
+
+// GELU, tanh form (Hendrycks and Gimpel): 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+  return 0.5f * x * (1.f + tanhf(u));
+}
+
+__global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_constant__ LinearParams p) {
+  constexpr int ST = kLinStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = sm;
+  uint8_t* sB = sA + ST * kLinABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + ST * kLinBBytes);  // [ST] stage loaded
+  uint64_t* empty = full + ST;                                          // [ST] stage consumed
+  uint64_t* acc_full = empty + ST;                                      // [2] accumulator complete
+  uint64_t* acc_empty = acc_full + 2;                                   // [2] accumulator read back
+  uint64_t* drain = acc_empty + 2;                                      // MMA abort path
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (p.d_in + 63) / 64;
+  // tiles of this CTA: t = blockIdx.x + i * gridDim.x
+  const int n_local = p.tiles > static_cast<int>(blockIdx.x)
+                          ? (p.tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                          : 0;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);  // every epilogue thread
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  auto tile_coords = [&](int i, int& b, int& r0, int& n0) {
+    const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    b = mt / p.m_tiles;
+    r0 = (mt % p.m_tiles) * 128;
+    n0 = nt * 256;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.x_map);
+      tma_prefetch_desc(&p.w_map);
+    }
+    int issued = 0;  // k chunks issued over all tiles
+    bool ok = true;
+    for (int i = 0; i < n_local && ok; ++i) {
+      int b, r0, n0;
+      tile_coords(i, b, r0, n0);
+      // rows 4 lane .. 4 lane + 3 of the tile (the ragged tail repeats the
+      // last row; its outputs are not stored)
+      int y[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        int r = r0 + 4 * lane + u;
+        r = r < p.R ? r : p.R - 1;
+        int idx = p.S != nullptr ? __ldg(p.S + static_cast<size_t>(b) * p.R + r) : r;
+        if (idx < 0 || idx >= p.N) {
+          raise_status(1 << 5);
+          idx = 0;
+        }
+        y[u] = b * p.N + idx;
+      }
+      for (int kc = 0; kc < nk; ++kc) {
+        const int g = i * nk + kc, s = g % ST;
+        if (g >= ST && !warp_wait(&empty[s], ((g / ST) - 1) & 1, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], kLinABytes + kLinBBytes);
+          tma_load_2d(sB + s * kLinBBytes, &p.w_map, &full[s], 64 * kc, n0);
+        }
+        __syncwarp();
+        tma_gather4(sA + s * kLinABytes + 4 * lane * 128, &p.x_map, &full[s], 64 * kc, y[0], y[1], y[2], y[3]);
+        issued = g + 1;
+      }
+    }
+    if ((!ok || abort_flag) && lane == 0) {
+      // let every copy this CTA started land before it exits
+      for (int g = issued - ST < 0 ? 0 : issued - ST; g < issued; ++g) mbar_wait_drain(&full[g % ST], (g / ST) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_bf16(128, 256, 0, 0);
+      bool ok = true;
+      for (int i = 0; i < n_local && ok; ++i) {
+        const int a = i & 1;
+        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) - 1) & 1, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tacc = tbase + 256u * a;
+        for (int kc = 0; kc < nk; ++kc) {
+          const int g = i * nk + kc, s = g % ST;
+          if (!mbar_wait(&full[s], (g / ST) & 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kLinABytes), b0 = smem_u32(sB + s * kLinBBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(tacc, make_sdesc(a0 + 32 * kk, 16, 1024, kSwizzle128B),
+                    make_sdesc(b0 + 32 * kk, 16, 1024, kSwizzle128B), idesc, (kc | kk) != 0 ? 1u : 0u);
+          umma_commit(&empty[s]);  // the stage may be refilled once these MMAs have read it
+        }
+        if (ok) umma_commit(&acc_full[a]);
+      }
+      if (!ok) {
+        // wait for every MMA this thread issued before TMEM is released
+        umma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3, row = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    for (int i = 0; i < n_local; ++i) {
+      const int a = i & 1;
+      if (!warp_wait(&acc_full[a], (i >> 1) & 1, &abort_flag)) break;
+      tc_fence_after();
+      int b, r0, n0;
+      tile_coords(i, b, r0, n0);
+      const int r = r0 + row;
+      const bool valid = r < p.R;
+      __nv_bfloat16* yrow = p.Y + (static_cast<size_t>(b) * p.R + (valid ? r : 0)) * p.d_out;
+      const uint32_t tacc = tbase + lane_addr + 256u * a;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tacc + 32 * c, v);
+        tmem_ld_wait32(v);
+        if (c == 7) {
+          // the whole accumulator is in registers or stored: release it
+          tc_fence_before();
+          mbar_arrive(&acc_empty[a]);
+        }
+        const int nc = n0 + 32 * c;
+        if (nc >= p.d_out) continue;
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float f0 = __uint_as_float(v[2 * e]), f1 = __uint_as_float(v[2 * e + 1]);
+          if (p.bias != nullptr) {
+            f0 += nc + 2 * e < p.d_out ? __ldg(p.bias + nc + 2 * e) : 0.f;
+            f1 += nc + 2 * e + 1 < p.d_out ? __ldg(p.bias + nc + 2 * e + 1) : 0.f;
+          }
+          if (p.act == 1) {
+            f0 = gelu_tanh_f(f0);
+            f1 = gelu_tanh_f(f1);
+          }
+          pk[e] = pack_bf16x2(f0, f1);
+        }
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (nc + 8 * u < p.d_out)
+              *reinterpret_cast<uint4*>(yrow + nc + 8 * u) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
+                                                                        pk[4 * u + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tbase, 512);
+}
+
+}  // namespace safe

@@ -17,12 +17,13 @@
 #include "cross_attn.cuh"
 #include "aux_kernels.cuh"
 #include "guidance.cuh"
+#include "linear.cuh"
 
 using namespace safe;
 
 namespace {
 
-constexpr int kAbiVersion = 4;
+constexpr int kAbiVersion = 5;
 constexpr float kLog2e = 1.4426950408889634f;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -90,6 +91,22 @@ bool encode_v_map(CUtensorMap* map, const void* base, int B, int rows, int H, in
 }
 
 // [B*N, H*d] 2-D view for tile::gather4 (box one row high).
+// 2-D bf16 matrix [outer, inner] (row pitch = inner), 128B swizzle; box
+// box_inner x box_outer (the row-wise layers' X, box 64 x 1 for gather4, and
+// W^T, box 64 x 256).
+bool encode_matrix_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                       uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_gather_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int c) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
@@ -621,6 +638,45 @@ safe_status safe_sensitivity_field(const float* scores, float* s, int B, int gri
   smooth_rows_kernel<<<grid, 256, 0, st>>>(p);
   smooth_cols_kernel<<<grid, 256, 0, st>>>(p);
   norm01_kernel<<<grid, 256, 0, st>>>(s, p.minmax, N);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- row-wise layers of the block
+safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const void* Wt, const float* bias, int act,
+                               void* Y, int B, int N, int d_in, int d_out, void* stream) {
+  if (!aligned16(X) || !aligned16(Wt) || !aligned16(Y)) return SAFE_ERR_INVALID_ARG;
+  if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u) != 0) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, 1) || (S != nullptr && (k < 1 || k > N))) return SAFE_ERR_INVALID_ARG;
+  if (d_in < 64 || d_in % 8 != 0 || d_out < 8 || d_out % 8 != 0 || (act != 0 && act != 1)) return SAFE_ERR_INVALID_ARG;
+  const int R = S != nullptr ? k : N;
+  const int64_t m_tiles = (R + 127) / 128, n_tiles = (d_out + 255) / 256;
+  const int64_t tiles = static_cast<int64_t>(B) * m_tiles * n_tiles;
+  if (tiles > INT_MAX) return SAFE_ERR_UNSUPPORTED;
+  LinearParams p{};
+  if (!encode_matrix_map(&p.x_map, X, static_cast<uint64_t>(d_in), static_cast<uint64_t>(B) * N, 64, 1) ||
+      !encode_matrix_map(&p.w_map, Wt, static_cast<uint64_t>(d_in), static_cast<uint64_t>(d_out), 64, 256))
+    return SAFE_ERR_CUDA;
+  p.S = S;
+  p.bias = bias;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.B = B;
+  p.N = N;
+  p.R = R;
+  p.d_in = d_in;
+  p.d_out = d_out;
+  p.act = act;
+  p.m_tiles = static_cast<int>(m_tiles);
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.tiles = static_cast<int>(tiles);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
+  });
+  if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
+  const int sms = device_sms();
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  linear_kernel<<<grid, kLinThreads, kLinSmem, as_stream(stream)>>>(p);
   return launch_status();
 }
 

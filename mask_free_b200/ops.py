@@ -49,6 +49,7 @@ _SIGS = {
     "safe_sensitivity_field": [_vp, _vp, _i, _i, _i, _f, _f, _vp, _sz, _vp],
     "safe_partition_indicator": [_vp, _i, _vp, _i, _i, _vp],
     "safe_sw_cfg": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _vp],
+    "safe_gather_linear": [_vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _vp],
 }
 _RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_attn_workspace_bytes": _sz, "safe_sensitivity_workspace_bytes": _sz,
              "safe_status_string": ctypes.c_char_p}
@@ -442,3 +443,32 @@ def sw_cfg(f_c, f_u, s, gamma_ctx: float, gamma_sens: float, out=None):
                                             float(gamma_ctx), float(gamma_sens), _stream()))
     return out
 
+
+
+_ACTS = {"none": 0, "gelu_tanh": 1}
+
+
+def gather_linear(X, Wt, S=None, bias=None, act="none", out=None):
+    """A row-wise layer of the row-selective block (Eq. (13), (15)):
+    Y[b, r, :] = act(X[b, S[b, r], :] W^T + bias); S = None: every row (the
+    dense block). X [B, N, d_in] bf16, Wt [d_out, d_in] bf16, S [B, k] int32,
+    bias [d_out] fp32, act "none" or "gelu_tanh". Returns [B, k or N, d_out]."""
+    _need(X, "X", torch.bfloat16, 3)
+    B, N, d_in = X.shape
+    dev = X.device
+    _need(Wt, "Wt", torch.bfloat16, 2, device=dev)
+    d_out = Wt.shape[0]
+    _need(Wt, "Wt", torch.bfloat16, 2, (d_out, d_in), dev)
+    k, R = 0, N
+    if S is not None:
+        _need(S, "S", torch.int32, 2, device=dev)
+        k = R = S.shape[1]
+        _need(S, "S", torch.int32, 2, (B, k), dev)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1, (d_out,), dev)
+    if act not in _ACTS:
+        raise ValueError(f"act must be one of {sorted(_ACTS)}, got {act!r}")
+    out = _out(out, "out", torch.bfloat16, (B, R, d_out), dev)
+    _check("safe_gather_linear", lib().safe_gather_linear(_p(X), _p(S), k, _p(Wt), _p(bias), _ACTS[act], _p(out), B,
+                                                          N, d_in, d_out, _stream()))
+    return out

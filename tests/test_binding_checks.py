@@ -88,6 +88,12 @@ def test_valid_calls_reach_the_abi_with_their_sizes(rec):
     assert _last(rec, "safe_sw_cfg")[4:8] == (2, B, N, 4)
     ops.mask_classify(torch.ones((B, 1, N, N), dtype=torch.bool), sync=False)
     _last(rec, "safe_mask_classify")
+    ops.gather_linear(t(B, N, 64), t(40, 64), S=S, bias=t(40, dtype=f32), act="gelu_tanh")
+    a = _last(rec, "safe_gather_linear")
+    assert a[2] == k and a[5] == 1 and a[7:11] == (B, N, 64, 40)
+    ops.gather_linear(t(B, N, 64), t(40, 64))
+    a = _last(rec, "safe_gather_linear")
+    assert a[1] is None and a[2] == 0 and a[5] == 0
 
 
 def _refused(fn, *args, **kw):
@@ -138,6 +144,13 @@ def test_mismatched_shapes_are_refused_before_any_launch(rec):
     _refused(ops.sw_cfg, fc, fc, t(B, N - 1, dtype=f32), 1.0, 5.0)
     _refused(ops.sw_cfg, fc, fc, t(B, N, dtype=f32), 1.0, 5.0, out=t(B, N, 4, dtype=bf16))
     _refused(ops.mask_classify, torch.ones((B, 1, N, N), dtype=torch.bool), result=t(4, dtype=torch.int64))
+    # row-wise layer: weight width, rows, bias, activation, output
+    X = t(B, N, 24)
+    _refused(ops.gather_linear, X, t(40, 32))
+    _refused(ops.gather_linear, X, t(40, 24), S=t(B + 1, k, dtype=i32))
+    _refused(ops.gather_linear, X, t(40, 24), bias=t(41, dtype=f32))
+    _refused(ops.gather_linear, X, t(40, 24), act="relu")
+    _refused(ops.gather_linear, X, t(40, 24), S=S, out=t(B, N, 40))
     assert rec.calls == []  # nothing reached the library
 
 
