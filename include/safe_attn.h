@@ -17,7 +17,8 @@
  *      image tensors Q, K, V, O, Kc, Vc    [B, N, H, d]
  *      compact row tensors (rows of S)     [B, k, H, d]
  *      text tensors Ky, Vy                 [B, M, H, d]
- *  - Supported head dims d: 64, 96, 128. `scale` is the logit scale (the
+ *      hidden states X (row-wise layers)   [B, N, d_in], weights W^T [d_out, d_in]
+ *  - Supported head dims d (attention): 64, 96, 128. `scale` is the logit scale (the
  *    paper uses 1/sqrt(d), Eq. (2)).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every
  *    call is asynchronous on `stream` unless it says "synchronises".
