@@ -10,8 +10,11 @@
  * ---------------------------------------
  *  - Pointers marked "device" are caller-owned device memory on the current
  *    CUDA device; pointers marked "host" are host memory. The library
- *    allocates no device memory and keeps no state between calls except the
- *    device status word (safe_get_device_status).
+ *    allocates no device memory. It keeps state between calls in two
+ *    places only: the device status word (safe_get_device_status) and the
+ *    fixed scratch array of the allocation-free entry point
+ *    safe_pcsp_topk_noalloc, which holds the last such call's per-head
+ *    partial scores.
  *  - bf16 tensors are passed as `const void*` / `void*` and must be 16-byte
  *    aligned and contiguous in the layouts stated (row-major, innermost last):
  *      image tensors Q, K, V, O, Kc, Vc    [B, N, H, d]
@@ -19,7 +22,8 @@
  *      text tensors Ky, Vy                 [B, M, H, d]
  *      hidden states X (row-wise layers)   [B, N, d_in], weights W^T [d_out, d_in]
  *  - Supported head dims d (attention): 64, 96, 128. `scale` is the logit scale (the
- *    paper uses 1/sqrt(d), Eq. (2)).
+ *    paper uses 1/sqrt(d), Eq. (2)); it must be finite and positive, else
+ *    SAFE_ERR_INVALID_ARG.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every
  *    call is asynchronous on `stream` unless it says "synchronises".
  *  - Errors: arguments are validated on the host before any launch and a
@@ -52,7 +56,7 @@ typedef enum {
 
 typedef enum { SAFE_BOOL = 0, SAFE_U8 = 1, SAFE_F32 = 2, SAFE_F16 = 3, SAFE_BF16 = 4 } safe_dtype;
 
-/* ABI version of this header (bumped on any signature or entry-point change): 5. */
+/* ABI version of this header (bumped on any signature or entry-point change): 6. */
 int safe_abi_version(void);
 const char* safe_status_string(int status);
 
@@ -315,10 +319,17 @@ safe_status safe_sw_cfg(const void* f_c, const void* f_u, const float* s, void* 
  *  Wt    device bf16 [d_out, d_in] (the weight of y = x W^T + b).
  *  bias  device fp32 [d_out] (4-byte aligned) or NULL.
  *  Y     device bf16 [B, k or N, d_out] (written; may not overlap X or Wt).
+ *  ws    device workspace of safe_gather_linear_workspace_bytes(B, k, d_in)
+ *        bytes (16-byte aligned; caller-owned, contents undefined after the
+ *        call), used with S only: the rows of S are first copied into it as
+ *        a compact [B, k, d_in] matrix, which the GEMM then reads by tiled
+ *        copies. NULL (or ws_bytes too small): the GEMM gathers the rows of
+ *        S itself, correct but slower. Ignored when S == NULL.
  *  d_in >= 64 and d_out >= 8, both multiples of 8; X, Wt, Y 16-byte aligned.
  */
+size_t safe_gather_linear_workspace_bytes(int B, int k, int d_in);
 safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const void* Wt, const float* bias, int act,
-                               void* Y, int B, int N, int d_in, int d_out, void* stream);
+                               void* Y, int B, int N, int d_in, int d_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Device status word: synchronises `stream`, writes to *h_status (host) the

@@ -7,7 +7,8 @@
 // of one (b, h) and pipelines them:
 //   warp 0      TMA producer: query tiles (dense rows, or rows of S via
 //               gather4) into a ring of QS shared-memory slots;
-//   warps 1, 2  MMA issuers, one per softmax warpgroup (even / odd tiles):
+//   warps 1, 2  MMA issuers, one per softmax warpgroup (even / odd tiles;
+//               the whole warp runs the loop, one elected lane issues):
 //               S = Q Ky^T (N = Lp = ceil32(valid_len)) into TMEM, then
 //               O = P Vy with P read from TMEM;
 //   warp 3      output store: the bf16 O tile, staged by the warpgroup in
@@ -274,7 +275,9 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
     const int g = warp - 1;
-    if (lane == 0) {
+    {
+      // the whole warp runs the issue loop; the elected lane issues
+      const uint32_t leader = elect_one_sync();
       const uint32_t tS = tbase + col_S(g), tO = tbase + col_O(g), tP = tbase + col_P(g);
       const uint32_t idS = make_idesc_bf16(128, Lp, 0, 0);
       constexpr uint32_t idPV = make_idesc_bf16(128, D, 0, 1);
@@ -287,24 +290,24 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2;
           const uint64_t bd = make_sdesc(aK + c * Mp * 128 + (kk & 3) * 32, 16, 8 * C::row_bytes(c), C::swizzle(c));
-          umma_ss(tS, kmajor_desc<D>(aQ, kk), bd, idS, kk > 0 ? 1u : 0u);
+          umma_ss_if(leader, tS, kmajor_desc<D>(aQ, kk), bd, idS, kk > 0 ? 1u : 0u);
         }
         if (L < Lp)  // padding keys -> -inf
-          umma_ss(tS, make_sdesc(smem_u32(sOnes), 16, 256, kSwizzle32B), make_sdesc(smem_u32(sBias), 16, 256, kSwizzle32B),
-                  idS, 1u);
-        umma_commit(&s_full[g]);
-        if (kSep || !has_o) umma_commit(&q_empty[i % QS]);
+          umma_ss_if(leader, tS, make_sdesc(smem_u32(sOnes), 16, 256, kSwizzle32B),
+                     make_sdesc(smem_u32(sBias), 16, 256, kSwizzle32B), idS, 1u);
+        umma_commit_if(leader, &s_full[g]);
+        if (kSep || !has_o) umma_commit_if(leader, &q_empty[i % QS]);
       };
       auto issue_PV = [&]() {
         for (int kk = 0; kk < Lp / 16; ++kk)
-          umma_ts(tO, tP + kk * 8, make_sdesc(aV + kk * 16 * 64, Mp * 64, 512, kSwizzle64B), idPV, kk > 0 ? 1u : 0u);
-        if (kSep) umma_commit(&pv_done[g]);
-        umma_commit(&o_full[g]);
+          umma_ts_if(leader, tO, tP + kk * 8, make_sdesc(aV + kk * 16 * 64, Mp * 64, 512, kSwizzle64B), idPV, kk > 0 ? 1u : 0u);
+        if (kSep) umma_commit_if(leader, &pv_done[g]);
+        umma_commit_if(leader, &o_full[g]);
       };
       if constexpr (kSep) {
         // per tile: the next S as soon as the softmax has loaded the
         // current one, then P V once P is written
-        bool ok = g < n_my && mbar_wait(&q_full[g % QS], (g / QS) & 1, &abort_flag);
+        bool ok = g < n_my && warp_wait(&q_full[g % QS], (g / QS) & 1, &abort_flag);
         if (ok) {
           tc_fence_after();
           issue_S(g);
@@ -312,14 +315,14 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         for (int i = g; ok && i < n_my; i += 2) {
           const int k = i >> 1;
           if (i + 2 < n_my) {
-            ok = mbar_wait(&q_full[(i + 2) % QS], ((i + 2) / QS) & 1, &abort_flag) &&
-                 mbar_wait(&s_free[g], k & 1, &abort_flag);
+            ok = warp_wait(&q_full[(i + 2) % QS], ((i + 2) / QS) & 1, &abort_flag) &&
+                 warp_wait(&s_free[g], k & 1, &abort_flag);
             if (!ok) break;
             tc_fence_after();
             issue_S(i + 2);
           }
           if (has_o) {
-            ok = mbar_wait(&p_full[g], k & 1, &abort_flag) && (k == 0 || mbar_wait(&t_free[g], (k - 1) & 1, &abort_flag));
+            ok = warp_wait(&p_full[g], k & 1, &abort_flag) && (k == 0 || warp_wait(&t_free[g], (k - 1) & 1, &abort_flag));
             if (!ok) break;
             tc_fence_after();
             issue_PV();
@@ -328,24 +331,24 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
       } else {
         for (int i = g; i < n_my; i += 2) {
           const int k = i >> 1;
-          if (!mbar_wait(&q_full[i % QS], (i / QS) & 1, &abort_flag)) break;
+          if (!warp_wait(&q_full[i % QS], (i / QS) & 1, &abort_flag)) break;
           // the previous tile of this warpgroup has released S (and, when S
           // reaches into the O columns, its output)
           if (k > 0) {
             uint64_t* prev = (has_o && Lp <= 128) ? &o_full[g] : &t_free[g];
-            if (!mbar_wait(prev, (k - 1) & 1, &abort_flag)) break;
+            if (!warp_wait(prev, (k - 1) & 1, &abort_flag)) break;
           }
           tc_fence_after();
           issue_S(i);
           if (!has_o) continue;
-          if (!mbar_wait(&p_full[g], k & 1, &abort_flag)) break;
-          if (k > 0 && !mbar_wait(&t_free[g], (k - 1) & 1, &abort_flag)) break;
+          if (!warp_wait(&p_full[g], k & 1, &abort_flag)) break;
+          if (k > 0 && !warp_wait(&t_free[g], (k - 1) & 1, &abort_flag)) break;
           tc_fence_after();
           issue_PV();
         }
       }
-      // every MMA this thread issued has completed before TMEM is released
-      umma_commit(&drained[g]);
+      // every MMA the leader issued has completed before TMEM is released
+      umma_commit_if(leader, &drained[g]);
       mbar_wait_drain(&drained[g], 0);
     }
   } else if (warp == 3) {

@@ -24,13 +24,21 @@
 //                the log-sum-exp.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
-// O1 [256+D,256+2D) and, for D <= 96, one 64-column P buffer after O1 shared
-// by the two tiles. With the separate P buffer the softmax releases S_t as
-// soon as it has loaded it, so S_t for the next key tile is computed while
-// the softmax is still exponentiating; the P buffer alternates strictly
-// P0_j, P1_j, P0_{j+1}, ... (each write waits for the other tile's previous
-// P V product). For D = 128 there is no room for it: P overwrites S_t and the
-// next S_t is issued after P_t V.
+// O1 [256+D,256+2D), then P (bf16 pairs, 64 columns for 128 keys):
+//   D = 64:  one P buffer per tile; each tile only waits for its own P V;
+//   D = 96:  one P buffer shared by the two tiles, written in strict
+//            alternation P0_j, P1_j, P0_{j+1}, ... (each write waits for the
+//            other tile's previous P V, which also orders the O rescale);
+//   D = 128: no room: P overwrites S_t and the next S_t follows P_t V.
+// With a separate P buffer the softmax releases S_t as soon as it has loaded
+// it, so S_t for the next key tile is computed while it exponentiates.
+//
+// The two tiles' softmax warps of one SM sub-partition (warps 4 + q and
+// 8 + q) share its exp unit and take turns on it (named barriers): one
+// exponentiates a whole key tile while the other stores P, waits for its next
+// S, loads it and takes the row max. The exponentials of a key tile run as
+// one pass of 128 independent instructions so that one warp keeps the unit
+// busy on its own.
 //
 // Online softmax in base 2: p = 2^(s*scale*log2(e) - m); O is only rescaled
 // when the running max grows by more than 8 (p stays below 2^8 otherwise).
@@ -38,12 +46,6 @@
 
 #include "sm100.cuh"
 
-// Pairs of probabilities whose 2^x is evaluated by the FMA-pipe polynomial
-// instead of the MUFU unit: bit i of the mask selects pair i of every
-// 16-pair (32-column) chunk of a row.
-#ifndef SAFE_EXP_EMU_MASK
-#define SAFE_EXP_EMU_MASK 0x0000u
-#endif
 
 namespace safe {
 
@@ -68,9 +70,14 @@ struct TileCfg {
   static constexpr int kVChunks = D / kVW;
   static constexpr uint32_t kVChunkBytes = 128u * kVW * 2u;
   static constexpr uint32_t kVSwizzle = kVW == 32 ? kSwizzle64B : kSwizzle128B;
-  // TMEM columns
+  // TMEM columns: O_t at kColO + t D; P_t at kColP (+ 64 t with one P
+  // buffer per tile) when P has a buffer of its own (kSepP), else in S_t
+  static constexpr bool kPerTileP = 256 + 2 * D + 128 <= 512;
   static constexpr bool kSepP = 256 + 2 * D + 64 <= 512;
   static constexpr uint32_t kColO = 256, kColP = 256 + 2 * D;
+  __host__ __device__ static constexpr uint32_t col_p(int t) {
+    return kSepP ? kColP + (kPerTileP ? 64u * t : 0u) : 128u * t;
+  }
 };
 
 // K-major operand (rows of a 128-row tile, contiguous along the head dim):
@@ -118,10 +125,14 @@ struct FlashParams {
   float2* ws_ml;          // [tail units][split][256] (running max in log2 units, row sum)
 };
 
-constexpr int kFlashThreads = 384;
-// Register split after setmaxnreg: warpgroup 0 (producer, MMA issuer) keeps
-// 104, the two softmax warpgroups get 200: 128*104 + 256*200 = 384*168, the
-// allocation the kernel is launched with (168 per thread).
+constexpr int kFlashThreads = 640;
+// Register split after setmaxnreg: warpgroup 0 (producer, MMA issuers)
+// keeps kFlashRegsControl, the four softmax warpgroups get
+// kFlashRegsSoftmax: 128 * 40 + 512 * 104 = 58368 <= 640 * 96, the
+// allocation the kernel is launched with (at most 96 per thread).
+constexpr uint32_t kFlashRegsControl = 40, kFlashRegsSoftmax = 104;
+// Shared by the cross-attention kernel (384 threads, 168 per thread at
+// launch): 128 * 104 + 256 * 200 = 384 * 168.
 constexpr uint32_t kRegsControl = 104, kRegsSoftmax = 200;
 
 template <int D>
@@ -327,7 +338,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   uint64_t* s_full = kv_empty + ST;  // [2] S_t computed
   uint64_t* s_free = s_full + 2;     // [2] S_t loaded by the softmax (separate-P mode)
   uint64_t* p_full = s_free + 2;     // [2] P_t written
-  uint64_t* pv_done = p_full + 2;    // [2] P_t V complete
+  uint64_t* pv_done = p_full + 2;    // [2] P_t V complete (separate-P mode)
   uint64_t* o_full = pv_done + 2;    // [2] last P_t V complete
   uint64_t* drain = o_full + 2;      // [2] per MMA issuer, abort path only
   uint64_t* k_ready = drain + 2;     // [ST] assembled mode: rows of S written into K_j (32 arrivals)
@@ -363,8 +374,8 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&s_free[t], 128);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&s_free[t], 256);  // both column halves of the tile's 128 rows
+      mbar_init(&p_full[t], 256);
       mbar_init(&pv_done[t], 1);
       mbar_init(&o_full[t], 1);
     }
@@ -379,7 +390,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   const uint32_t tbase = *tmem_slot;
 
   if (warp < 4) {
-    regs_dealloc<kRegsControl>();
+    regs_dealloc<kFlashRegsControl>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {
@@ -444,8 +455,11 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       // ---------------------------------------------------------- MMA issuers
       // separate-P mode: warp 1 issues tile 0's MMAs and warp 2 tile 1's
       // (tcgen05.commit tracks the issuing thread's MMAs, so each issuer
-      // signals its own tile); aliased mode: warp 1 issues both tiles.
-      if (lane == 0) {
+      // signals its own tile); aliased mode: warp 1 issues both tiles. Each
+      // issuing warp runs its loop with all lanes and one elected lane issues.
+      {
+        // the whole warp runs the issue loop; the elected lane issues
+        const uint32_t leader = elect_one_sync();
         const int mt = warp - 1;  // tile of this issuer (separate-P mode)
         constexpr uint32_t idS = make_idesc_bf16(128, 128, 0, 0);
         constexpr uint32_t idPV = make_idesc_bf16(128, D, 0, 1);
@@ -453,7 +467,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
         // TMEM column of S_t, O_t and P_t (t = 0, 1)
         auto tS = [&](int t) -> uint32_t { return tbase + 128u * t; };
         auto tO = [&](int t) -> uint32_t { return tbase + C::kColO + static_cast<uint32_t>(D) * t; };
-        auto tP = [&](int t) -> uint32_t { return kSepP ? tbase + C::kColP : tbase + 128u * t; };
+        auto tP = [&](int t) -> uint32_t { return tbase + C::col_p(t); };
         // stage barriers the MMAs wait on: the TMA copy, or, with assembled
         // keys, the rows of S written over it
         uint64_t* k_in = kAsm ? k_ready : k_full;
@@ -475,7 +489,8 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
           const uint32_t so = static_cast<uint32_t>((s * TB) >> 4);
           const uint64_t dq = t == 0 ? dQ0 : dQ1;
 #pragma unroll
-          for (int kk = 0; kk < KS; ++kk) umma_ss(tS(t), kdesc(dq, kk, 0), kdesc(dK, kk, so), idS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < KS; ++kk)
+            umma_ss_if(leader, tS(t), kdesc(dq, kk, 0), kdesc(dK, kk, so), idS, kk > 0 ? 1u : 0u);
         };
         // O_t (+)= P_t V: 8 steps of 16 keys, one N = D instruction each
         auto issue_PV = [&](int t, int s, int j) {
@@ -483,72 +498,73 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t v = static_cast<uint32_t>(dV) + so + ((kk * 16 * C::kVW * 2) >> 4);
-            umma_ts(tO(t), tP(t) + kk * 8, (dV & 0xFFFFFFFF00000000ull) | v, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts_if(leader, tO(t), tP(t) + kk * 8, (dV & 0xFFFFFFFF00000000ull) | v, idPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
           }
         };
-        bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&k_in[0], 0, &abort_flag);
+        bool ok = warp_wait(q_full, 0, &abort_flag) && warp_wait(&k_in[0], 0, &abort_flag);
         if (ok) {
           tc_fence_after();
           if constexpr (kSepP) {
             // per tile: the next S as soon as the softmax has loaded the
             // current one, then P V once P is written
             issue_S(mt, 0);
-            umma_commit(&s_full[mt]);
+            umma_commit_if(leader, &s_full[mt]);
             for (int j = 0; j < n_kv && ok; ++j) {
               const int s = j % ST;
               if (j + 1 < n_kv) {
                 const int s1 = (j + 1) % ST;
-                ok = mbar_wait(&k_in[s1], ((j + 1) / ST) & 1, &abort_flag) &&
-                     mbar_wait(&s_free[mt], j & 1, &abort_flag);
+                ok = warp_wait(&k_in[s1], ((j + 1) / ST) & 1, &abort_flag) &&
+                     warp_wait(&s_free[mt], j & 1, &abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 issue_S(mt, s1);
-                umma_commit(&s_full[mt]);
+                umma_commit_if(leader, &s_full[mt]);
               }
-              ok = mbar_wait(&v_in[s], (j / ST) & 1, &abort_flag) && mbar_wait(&p_full[mt], j & 1, &abort_flag);
+              ok = warp_wait(&v_in[s], (j / ST) & 1, &abort_flag) && warp_wait(&p_full[mt], j & 1, &abort_flag);
               if (!ok) break;
               tc_fence_after();
               issue_PV(mt, s, j);
-              umma_commit(&pv_done[mt]);
-              umma_commit(&kv_empty[s]);  // this tile no longer reads K_j, V_j
-              if (j + 1 == n_kv) umma_commit(&o_full[mt]);
+              umma_commit_if(leader, &pv_done[mt]);
+              umma_commit_if(leader, &kv_empty[s]);  // this tile no longer reads K_j, V_j
+              if (j + 1 == n_kv) umma_commit_if(leader, &o_full[mt]);
             }
           } else {
           issue_S(0, 0);
-          umma_commit(&s_full[0]);
+          umma_commit_if(leader, &s_full[0]);
           issue_S(1, 0);
-          umma_commit(&s_full[1]);
+          umma_commit_if(leader, &s_full[1]);
           for (int j = 0; j < n_kv && ok; ++j) {
             const int s = j % ST;
             {
               // P overwrites S_t: the next S_t follows P_t V
-              ok = mbar_wait(&v_in[s], (j / ST) & 1, &abort_flag);
+              ok = warp_wait(&v_in[s], (j / ST) & 1, &abort_flag);
               for (int t = 0; t < 2 && ok; ++t) {
-                ok = mbar_wait(&p_full[t], j & 1, &abort_flag);
+                ok = warp_wait(&p_full[t], j & 1, &abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 issue_PV(t, s, j);
                 if (j + 1 < n_kv) {
                   const int s1 = (j + 1) % ST;
                   if (t == 0) {
-                    ok = mbar_wait(&k_in[s1], ((j + 1) / ST) & 1, &abort_flag);
+                    ok = warp_wait(&k_in[s1], ((j + 1) / ST) & 1, &abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                   }
                   issue_S(t, s1);
-                  umma_commit(&s_full[t]);
+                  umma_commit_if(leader, &s_full[t]);
                 } else {
-                  umma_commit(&o_full[t]);
+                  umma_commit_if(leader, &o_full[t]);
                 }
               }
             }
-            if (ok) umma_commit(&kv_empty[s]);
+            if (ok) umma_commit_if(leader, &kv_empty[s]);
           }
           }
         }
         if (!ok) {
-          // wait for every MMA this thread issued before TMEM is released
-          umma_commit(&drain[warp - 1]);
+          // wait for every MMA the leader issued before TMEM is released
+          umma_commit_if(leader, &drain[warp - 1]);
           mbar_wait_drain(&drain[warp - 1], 0);
         }
       }
@@ -557,44 +573,94 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       assemble_current_rows<D>(p, sK, sV, k_full, v_full, k_ready, v_ready, b, h, kv0, n_kv, &abort_flag);
     }
   } else {
-    regs_alloc<kRegsSoftmax>();
+    regs_alloc<kFlashRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 4) >> 2;
+    // Warp 4 + 4 g + q, g = 2 t + hf: query rows 32 q .. 32 q + 31 of tile
+    // t (TMEM lanes of sub-partition q), keys 64 hf .. 64 hf + 63 of each key
+    // tile (the column half hf of S and of P) and columns hf D/2 .. of O.
+    const int g = (warp - 4) >> 2, t = g >> 1, hf = g & 1;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tbase + lane_addr + t * 128;
-    const uint32_t tO = tbase + lane_addr + C::kColO + t * D;
-    const uint32_t tP = kSepP ? tbase + lane_addr + C::kColP : tS;
+    const uint32_t tS = tbase + lane_addr + t * 128 + 64 * hf;
+    constexpr int DH = D / 2;  // O columns of one half
+    const uint32_t tO = tbase + lane_addr + C::kColO + t * D + DH * hf;
+    const uint32_t tP = tbase + lane_addr + C::col_p(t) + 32 * hf;
     const int q_row = q_base + t * 128 + row;
     const float sl2 = p.scale_log2;
-    // valid keys in this CTA's last tile (fewer than 128 only in the global last tile)
-    const int tail = kv1 == n_kv_all ? p.N - (n_kv_all - 1) * 128 : 128;
+    // valid keys of this half in this CTA's last key tile (fewer than 64
+    // only in the global last tile)
+    const int tail = (kv1 == n_kv_all ? p.N - (n_kv_all - 1) * 128 : 128) - 64 * hf;
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!warp_wait(&s_full[t], j & 1, &abort_flag)) {
-        ok = false;
-        break;
+    // The four softmax warps of one SM sub-partition share its exp unit: the
+    // two column halves of tile 0 exponentiate together, then the two of
+    // tile 1, and so on, each pair loading S, taking its half-row max and
+    // storing P while the other pair exponentiates. Named barrier 1 + 2q + t
+    // is "tile t may exponentiate" (128 threads: the pair that waits and the
+    // pair that hands over); it also publishes the half-row maxima, which
+    // each half writes to shared memory before it waits. Every warp takes
+    // every barrier step on every path (an abort only skips the work).
+    const uint32_t bar_mine = 1 + 2 * quarter + t, bar_other = 1 + 2 * quarter + (1 - t);
+    __shared__ float half_max[2][2][2][128];  // [step parity][tile][half][row]
+    // store this half of P_t of key tile j (32 bf16 pairs in pk) and rescale
+    // this half of O_t first when the running max grew
+    auto store_p = [&](int j, const uint32_t* pk, bool need, float alpha) {
+      if constexpr (kSepP) {
+        // the P buffer is free and O_t idle: one buffer per tile: this
+        // tile's previous P V is complete; shared buffer: the other tile's
+        // previous P V (P0_j after P1_{j-1} V, P1_j after P0_j V; the
+        // other tile's write waited for this tile's previous P V)
+        bool w = true;
+        if (C::kPerTileP || t == 0) {
+          if (j > 0) w = warp_wait(&pv_done[C::kPerTileP ? t : 1], (j - 1) & 1, &abort_flag);
+        } else {
+          w = warp_wait(&pv_done[0], j & 1, &abort_flag);
+        }
+        if (!w) {
+          ok = false;
+          return;
+        }
+        tc_fence_after();
       }
+      // (aliased mode: O_t is idle because P_t V of the previous step
+      // completed before S_t of this step was committed)
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < DH / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16 * c, o);
+          tmem_ld_wait16(o);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16(tO + 16 * c, o);
+        }
+      }
+      tmem_st16(tP, pk);
+      tmem_st16(tP + 16, pk + 16);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    };
+    if (t == 1) named_bar_arrive(bar_other, 128);  // tile 0 goes first
+    for (int j = 0; j < n_kv; ++j) {
+      // After an abort the arithmetic still runs (on whatever TMEM holds)
+      // but no wait, arrival or store is made; the barrier steps stay.
+      if (ok) ok = warp_wait(&s_full[t], j & 1, &abort_flag);
       tc_fence_after();
-      uint32_t sr[128];
+      uint32_t sr[64];
       tmem_ld32(tS + 0, sr);
       tmem_ld32(tS + 32, sr + 32);
-      tmem_ld32(tS + 64, sr + 64);
-      tmem_ld32(tS + 96, sr + 96);
       tmem_ld_wait32(sr);
       tmem_ld_wait32(sr + 32);
-      tmem_ld_wait32(sr + 64);
-      tmem_ld_wait32(sr + 96);
-      if constexpr (kSepP) {
-        // S_t is in registers: the MMA issuer may overwrite it
+      if (kSepP && ok) {
+        // this half of S_t is in registers: the MMA issuer may overwrite it
         tc_fence_before();
         mbar_arrive(&s_free[t]);
       }
-      if (j == n_kv - 1 && tail < 128) {
+      if (j == n_kv - 1 && tail < 64) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c >= tail) sr[c] = __float_as_uint(-INFINITY);
       }
       float mx0 = fmax3(__uint_as_float(sr[0]), __uint_as_float(sr[1]), __uint_as_float(sr[2]));
@@ -602,15 +668,19 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       float mx2 = fmax3(__uint_as_float(sr[6]), __uint_as_float(sr[7]), __uint_as_float(sr[8]));
       float mx3 = fmax3(__uint_as_float(sr[9]), __uint_as_float(sr[10]), __uint_as_float(sr[11]));
 #pragma unroll
-      for (int c = 12; c < 124; c += 8) {
+      for (int c = 12; c < 60; c += 8) {
         mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
         mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
         mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
         mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
       }
-      mx0 = fmax3(mx0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
-      mx1 = fmax3(mx1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
-      const float m_cand = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+      mx0 = fmax3(mx0, __uint_as_float(sr[60]), __uint_as_float(sr[61]));
+      mx1 = fmax3(mx1, __uint_as_float(sr[62]), __uint_as_float(sr[63]));
+      const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+      half_max[j & 1][t][hf][row] = mx;
+      // ---- this tile's turn on the exp unit (and the other half's maximum)
+      named_bar_sync(bar_mine, 128);
+      const float m_cand = fmaxf(mx, half_max[j & 1][t][hf ^ 1][row]) * sl2;
       float alpha = 1.f;
       bool need = false;
       if (j == 0) {
@@ -622,83 +692,60 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
           m_use = m_cand;
         }
       }
-      // probabilities (bf16 pairs) and the row sum
+      // probabilities: x = s scale log2(e) - m, then 2^x as one pass of 64
+      // independent exponentials, then the row sum and the bf16 pairs
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m_use, -m_use);
+      float x[64];
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm2),
+                  x[2 * i], x[2 * i + 1]);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) x[c] = ex2_approx(x[c]);
+      uint32_t pk[32];
       uint64_t acc0 = 0, acc1 = 0;  // packed row sums (bit pattern 0 = +0.0f)
-      uint32_t pk[64];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm2);
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        uint64_t e2;
-        if ((SAFE_EXP_EMU_MASK >> (i & 15)) & 1u)
-          e2 = exp2_poly_f2(x0, x1);
-        else
-          e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      for (int i = 0; i < 32; ++i) {
+        const uint64_t e2 = f2_pack(x[2 * i], x[2 * i + 1]);
         if (i & 1) acc1 = f2_add(acc1, e2); else acc0 = f2_add(acc0, e2);
-        float a, bb;
-        f2_unpack(e2, a, bb);
-        pk[i] = pack_bf16x2(a, bb);
+        pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
       }
-      if constexpr (kSepP) {
-        // P buffer turn: P0_j follows P1_{j-1} V, P1_j follows P0_j V. That
-        // wait also orders this tile's previous P V before the O rescale.
-        bool turn = true;
-        if (t == 0 && j > 0) turn = warp_wait(&pv_done[1], (j - 1) & 1, &abort_flag);
-        if (t == 1) turn = warp_wait(&pv_done[0], j & 1, &abort_flag);
-        if (!turn) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
-      // (aliased mode: O_t is idle because P_t V of the previous step
-      // completed before S_t of this step was committed)
-      if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(tO + 16 * c, o);
-          tmem_ld_wait16(o);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(tO + 16 * c, o);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      // ---- hand the exp unit to the other tile
+      if (t == 0 || j + 1 < n_kv) named_bar_arrive(bar_other, 128);
+      if (ok) store_p(j, pk, need, alpha);
       float s0, s1, s2, s3;
       f2_unpack(acc0, s0, s1);
       f2_unpack(acc1, s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
     }
+    // the row sum is the sum of the two halves' sums (same running max)
+    __shared__ float half_sum[2][2][128];
+    half_sum[t][hf][row] = l;
+    named_bar_sync(9, 512);
+    l = half_sum[t][0][row] + half_sum[t][1][row];
     const bool have_o = ok && warp_wait(&o_full[t], 0, &abort_flag);
     if (have_o) tc_fence_after();
     const bool valid = q_row < p.n_q;
-    __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.n_q + (valid ? q_row : 0)) * p.H + h) * D;
+    __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.n_q + (valid ? q_row : 0)) * p.H + h) * D + DH * hf;
     if (have_o && !partial) {
       const float inv_l = 1.f / l;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * c, o);
-        tmem_ld_wait32(o);
-        uint32_t pk[16];
+      for (int c = 0; c < DH / 16; ++c) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16 * c, o);
+        tmem_ld_wait16(o);
+        uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
           pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      if (valid && p.lse != nullptr)
+      if (valid && hf == 0 && p.lse != nullptr)
         p.lse[(static_cast<size_t>(b) * p.H + h) * p.n_q + q_row] = (m_use + __log2f(l)) * 0.69314718055994531f;
     }
     if (partial) {
@@ -706,19 +753,19 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
       // running max and sum (flash_merge_kernel combines the parts)
       const size_t slot0 = static_cast<size_t>(tail_u) * p.split * 256 + t * 128 + row;
       if (have_o) {
-        float* po = p.ws_o + (slot0 + static_cast<size_t>(part) * 256) * D;
+        float* po = p.ws_o + (slot0 + static_cast<size_t>(part) * 256) * D + DH * hf;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_ld_wait32(o);
+        for (int c = 0; c < DH / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16 * c, o);
+          tmem_ld_wait16(o);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            reinterpret_cast<float4*>(po + 32 * c)[v] =
+          for (int v = 0; v < 4; ++v)
+            reinterpret_cast<float4*>(po + 16 * c)[v] =
                 make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]), __uint_as_float(o[4 * v + 2]),
                             __uint_as_float(o[4 * v + 3]));
         }
-        p.ws_ml[slot0 + static_cast<size_t>(part) * 256] = make_float2(m_use, l);
+        if (hf == 0) p.ws_ml[slot0 + static_cast<size_t>(part) * 256] = make_float2(m_use, l);
       }
     }
   }

@@ -9,11 +9,12 @@
 // Persistent kernel: one CTA per SM walks the 128 x 256 output tiles
 // t = blockIdx.x, blockIdx.x + gridDim.x, ... (the column tile fastest, so
 // CTAs running at the same time share their gathered rows of X through L2).
-//   warp 0     producer: per 64-wide K chunk, the 128 rows of X by TMA
-//              gather4 (lane l copies rows 4l .. 4l + 3) and the 256 x 64
-//              tile of W by one tiled copy, both K-major with the 128B
-//              swizzle, into a 4-stage ring
-//   warp 1     MMA issuer: tcgen05.mma M = 128, N = 256, K = 16 into one of
+//   warp 0     producer: per 64-wide K chunk, the 128 rows of X (rows of
+//              S: TMA gather4, lane l copies rows 4l .. 4l + 3; every row:
+//              one tiled copy) and the 256 x 64 tile of W by one tiled copy,
+//              both K-major with the 128B swizzle, into a 4-stage ring
+//   warp 1     MMA issuer (the whole warp runs the loop, one elected lane
+//              issues): tcgen05.mma M = 128, N = 256, K = 16 into one of
 //              two 256-column TMEM accumulators (tile i uses buffer i & 1)
 //   warp 2     TMEM allocation
 //   warps 4..7 epilogue: tcgen05.ld of the accumulator (TMEM lane = row of
@@ -30,6 +31,7 @@ namespace safe {
 
 struct LinearParams {
   CUtensorMap x_map;    // 2-D [B*N, d_in], box 64 x 1 (gather4)
+  CUtensorMap xt_map;   // 2-D [B*N, d_in], box 64 x 128 (every row: one tiled copy)
   CUtensorMap w_map;    // 2-D [d_out, d_in], box 64 x 256
   const int32_t* S;     // [B, R] rows of X, or null (rows 0 .. R-1)
   const float* bias;    // [d_out] or null
@@ -50,6 +52,26 @@ constexpr int kLinSmem = 1024 + kLinStages * (kLinABytes + kLinBBytes) + 256;
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
   return 0.5f * x * (1.f + tanhf(u));
+}
+
+// Xg[b, r, :] = X[b, S[b, r], :] for r < k, one warp per row, 16-byte
+// units (d_in is a multiple of 8). An index outside [0, N) is flagged and
+// row 0 is copied instead, as the gathering GEMM does.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ S,
+                                                          uint4* __restrict__ Xg, int B, int N, int k,
+                                                          int units_per_row) {
+  const int lane = threadIdx.x & 31;
+  const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (w >= static_cast<long long>(B) * k) return;
+  const int b = static_cast<int>(w / k), r = static_cast<int>(w % k);
+  int idx = __ldg(S + static_cast<size_t>(b) * k + r);
+  if (idx < 0 || idx >= N) {
+    if (lane == 0) raise_status(1 << 5);
+    idx = 0;
+  }
+  const uint4* src = X + (static_cast<size_t>(b) * N + idx) * units_per_row;
+  uint4* dst = Xg + (static_cast<size_t>(b) * k + r) * units_per_row;
+  for (int u = lane; u < units_per_row; u += 32) dst[u] = __ldg(src + u);
 }
 
 __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_constant__ LinearParams p) {
@@ -103,7 +125,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.x_map);
+      tma_prefetch_desc(p.S != nullptr ? &p.x_map : &p.xt_map);
       tma_prefetch_desc(&p.w_map);
     }
     int issued = 0;  // k chunks issued over all tiles
@@ -134,9 +156,14 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], kLinABytes + kLinBBytes);
           tma_load_2d(sB + s * kLinBBytes, &p.w_map, &full[s], 64 * kc, n0);
+          // every row: rows r0 .. r0 + 127 of sample b in one copy (rows
+          // past the sample's end are other samples' rows or the zero fill
+          // past the tensor; their outputs are not stored)
+          if (p.S == nullptr) tma_load_2d(sA + s * kLinABytes, &p.xt_map, &full[s], 64 * kc, b * p.N + r0);
         }
         __syncwarp();
-        tma_gather4(sA + s * kLinABytes + 4 * lane * 128, &p.x_map, &full[s], 64 * kc, y[0], y[1], y[2], y[3]);
+        if (p.S != nullptr)
+          tma_gather4(sA + s * kLinABytes + 4 * lane * 128, &p.x_map, &full[s], 64 * kc, y[0], y[1], y[2], y[3]);
         issued = g + 1;
       }
     }
@@ -146,38 +173,38 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_bf16(128, 256, 0, 0);
-      bool ok = true;
-      for (int i = 0; i < n_local && ok; ++i) {
-        const int a = i & 1;
-        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) - 1) & 1, &abort_flag)) {
+    const uint32_t leader = elect_one_sync();
+    constexpr uint32_t idesc = make_idesc_bf16(128, 256, 0, 0);
+    bool ok = true;
+    for (int i = 0; i < n_local && ok; ++i) {
+      const int a = i & 1;
+      if (i >= 2 && !warp_wait(&acc_empty[a], ((i >> 1) - 1) & 1, &abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tacc = tbase + 256u * a;
+      for (int kc = 0; kc < nk; ++kc) {
+        const int g = i * nk + kc, s = g % ST;
+        if (!warp_wait(&full[s], (g / ST) & 1, &abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t tacc = tbase + 256u * a;
-        for (int kc = 0; kc < nk; ++kc) {
-          const int g = i * nk + kc, s = g % ST;
-          if (!mbar_wait(&full[s], (g / ST) & 1, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * kLinABytes), b0 = smem_u32(sB + s * kLinBBytes);
+        const uint32_t a0 = smem_u32(sA + s * kLinABytes), b0 = smem_u32(sB + s * kLinBBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_ss(tacc, make_sdesc(a0 + 32 * kk, 16, 1024, kSwizzle128B),
-                    make_sdesc(b0 + 32 * kk, 16, 1024, kSwizzle128B), idesc, (kc | kk) != 0 ? 1u : 0u);
-          umma_commit(&empty[s]);  // the stage may be refilled once these MMAs have read it
-        }
-        if (ok) umma_commit(&acc_full[a]);
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ss_if(leader, tacc, make_sdesc(a0 + 32 * kk, 16, 1024, kSwizzle128B),
+                     make_sdesc(b0 + 32 * kk, 16, 1024, kSwizzle128B), idesc, (kc | kk) != 0 ? 1u : 0u);
+        umma_commit_if(leader, &empty[s]);  // the stage may be refilled once these MMAs have read it
       }
-      if (!ok) {
-        // wait for every MMA this thread issued before TMEM is released
-        umma_commit(drain);
-        mbar_wait_drain(drain, 0);
-      }
+      if (ok) umma_commit_if(leader, &acc_full[a]);
+    }
+    if (!ok) {
+      // wait for every MMA the leader issued before TMEM is released
+      umma_commit_if(leader, drain);
+      if (leader) mbar_wait_drain(drain, 0);
+      __syncwarp();
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue

@@ -23,7 +23,7 @@ using namespace safe;
 
 namespace {
 
-constexpr int kAbiVersion = 5;
+constexpr int kAbiVersion = 6;
 constexpr float kLog2e = 1.4426950408889634f;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -31,6 +31,11 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool supported_d(int d) { return d == 64 || d == 96 || d == 128; }
+
+// The attention kernels take each row's maximum of the unscaled logits and
+// scale it afterwards, which is the row's largest scaled logit only for a
+// positive scale; padding keys are masked with -inf before scaling.
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
 
 safe_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? SAFE_OK : SAFE_ERR_CUDA;
@@ -429,7 +434,7 @@ size_t safe_attn_workspace_bytes(int B, int n_q, int N, int H, int d) {
 safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O, float* lse, int B, int N, int H,
                            int d, float scale, void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SAFE_ERR_INVALID_ARG;
-  if (!sizes_ok(B, N, H) || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || !scale_ok(scale)) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
   for (int c = 0; c < nchunks(d); ++c) {
@@ -453,7 +458,7 @@ safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k
                            void* O_S, float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
                            void* stream) {
   if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O_S)) return SAFE_ERR_INVALID_ARG;
-  if (!sizes_ok(B, N, H) || k < 1 || k > N || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || k < 1 || k > N || !scale_ok(scale)) return SAFE_ERR_INVALID_ARG;
   if (!q_compact && S == nullptr) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
@@ -468,7 +473,7 @@ safe_status safe_srsu_attn_assembled(const void* Q, int q_compact, const int32_t
   if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O_S) || !aligned16(Kcur) ||
       !aligned16(Vcur) || S == nullptr)
     return SAFE_ERR_INVALID_ARG;
-  if (!sizes_ok(B, N, H) || k < 1 || k > N || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || k < 1 || k > N || !scale_ok(scale)) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
   if (!fill_srsu(p, Q, q_compact, S, k, Kc, Vc, O_S, lse, B, N, H, d, scale)) return SAFE_ERR_CUDA;
@@ -483,7 +488,7 @@ safe_status safe_attn_cross(const void* Q, const int32_t* q_idx, int nq, const v
                             void* stream) {
   if (!aligned16(Q) || !aligned16(Ky) || !aligned16(Vy) || !aligned16(O) || valid_len == nullptr)
     return SAFE_ERR_INVALID_ARG;
-  if (!sizes_ok(B, N, H) || M < 1 || !std::isfinite(scale)) return SAFE_ERR_INVALID_ARG;
+  if (!sizes_ok(B, N, H) || M < 1 || !scale_ok(scale)) return SAFE_ERR_INVALID_ARG;
   if (q_idx == nullptr ? nq != N : (nq < 1 || nq > N)) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d) || M > 256) return SAFE_ERR_UNSUPPORTED;
   CrossParams p;
@@ -510,7 +515,7 @@ safe_status safe_pcsp_topk(const void* Q, const void* Ky, const int32_t* valid_l
   if (k > 0 && S == nullptr) return SAFE_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   if (Q != nullptr) {
-    if (!aligned16(Q) || !aligned16(Ky) || valid_len == nullptr || M < 1 || !std::isfinite(scale))
+    if (!aligned16(Q) || !aligned16(Ky) || valid_len == nullptr || M < 1 || !scale_ok(scale))
       return SAFE_ERR_INVALID_ARG;
     if (!supported_d(d) || M > 256) return SAFE_ERR_UNSUPPORTED;
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 ||
@@ -538,7 +543,7 @@ safe_status safe_attn_cross_pcsp(const void* Q, const void* Ky, const void* Vy, 
                                  size_t ws_bytes, void* stream) {
   if (!aligned16(Q) || !aligned16(Ky) || !aligned16(Vy) || !aligned16(O) || valid_len == nullptr || scores == nullptr)
     return SAFE_ERR_INVALID_ARG;
-  if (!sizes_ok(B, N, H) || M < 1 || !std::isfinite(scale) || k < 0 || k > N || (k > 0 && S == nullptr))
+  if (!sizes_ok(B, N, H) || M < 1 || !scale_ok(scale) || k < 0 || k > N || (k > 0 && S == nullptr))
     return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d) || M > 256) return SAFE_ERR_UNSUPPORTED;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < safe_pcsp_workspace_bytes(B, N, H))
@@ -642,18 +647,36 @@ safe_status safe_sensitivity_field(const float* scores, float* s, int B, int gri
 }
 
 // ---------------------------------------------------------------- row-wise layers of the block
+size_t safe_gather_linear_workspace_bytes(int B, int k, int d_in) {
+  if (B < 1 || k < 1 || d_in < 1) return 0;
+  return static_cast<size_t>(B) * k * d_in * 2;
+}
+
 safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const void* Wt, const float* bias, int act,
-                               void* Y, int B, int N, int d_in, int d_out, void* stream) {
+                               void* Y, int B, int N, int d_in, int d_out, void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(X) || !aligned16(Wt) || !aligned16(Y)) return SAFE_ERR_INVALID_ARG;
   if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u) != 0) return SAFE_ERR_INVALID_ARG;
   if (!sizes_ok(B, N, 1) || (S != nullptr && (k < 1 || k > N))) return SAFE_ERR_INVALID_ARG;
   if (d_in < 64 || d_in % 8 != 0 || d_out < 8 || d_out % 8 != 0 || (act != 0 && act != 1)) return SAFE_ERR_INVALID_ARG;
+  if (S != nullptr && aligned16(ws) && ws_bytes >= safe_gather_linear_workspace_bytes(B, k, d_in)) {
+    // the rows of S as a compact [B, k, d_in] matrix, then the GEMM over
+    // every row of it (tiled operand copies instead of per-row gathers)
+    const long long rows = static_cast<long long>(B) * k;
+    if ((rows + 7) / 8 > INT_MAX) return SAFE_ERR_UNSUPPORTED;
+    gather_rows_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, as_stream(stream)>>>(
+        static_cast<const uint4*>(X), S, static_cast<uint4*>(ws), B, N, k, d_in / 8);
+    if (cudaGetLastError() != cudaSuccess) return SAFE_ERR_CUDA;
+    X = ws;
+    N = k;
+    S = nullptr;
+  }
   const int R = S != nullptr ? k : N;
   const int64_t m_tiles = (R + 127) / 128, n_tiles = (d_out + 255) / 256;
   const int64_t tiles = static_cast<int64_t>(B) * m_tiles * n_tiles;
   if (tiles > INT_MAX) return SAFE_ERR_UNSUPPORTED;
   LinearParams p{};
   if (!encode_matrix_map(&p.x_map, X, static_cast<uint64_t>(d_in), static_cast<uint64_t>(B) * N, 64, 1) ||
+      !encode_matrix_map(&p.xt_map, X, static_cast<uint64_t>(d_in), static_cast<uint64_t>(B) * N, 64, 128) ||
       !encode_matrix_map(&p.w_map, Wt, static_cast<uint64_t>(d_in), static_cast<uint64_t>(d_out), 64, 256))
     return SAFE_ERR_CUDA;
   p.S = S;

@@ -49,9 +49,11 @@ _SIGS = {
     "safe_sensitivity_field": [_vp, _vp, _i, _i, _i, _f, _f, _vp, _sz, _vp],
     "safe_partition_indicator": [_vp, _i, _vp, _i, _i, _vp],
     "safe_sw_cfg": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _vp],
-    "safe_gather_linear": [_vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _vp],
+    "safe_gather_linear_workspace_bytes": [_i, _i, _i],
+    "safe_gather_linear": [_vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _sz, _vp],
 }
 _RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_attn_workspace_bytes": _sz, "safe_sensitivity_workspace_bytes": _sz,
+             "safe_gather_linear_workspace_bytes": _sz,
              "safe_status_string": ctypes.c_char_p}
 
 
@@ -448,11 +450,17 @@ def sw_cfg(f_c, f_u, s, gamma_ctx: float, gamma_sens: float, out=None):
 _ACTS = {"none": 0, "gelu_tanh": 1}
 
 
-def gather_linear(X, Wt, S=None, bias=None, act="none", out=None):
+def gather_linear_workspace_bytes(B: int, k: int, d_in: int) -> int:
+    return int(lib().safe_gather_linear_workspace_bytes(B, k, d_in))
+
+
+def gather_linear(X, Wt, S=None, bias=None, act="none", out=None, ws=None):
     """A row-wise layer of the row-selective block (Eq. (13), (15)):
     Y[b, r, :] = act(X[b, S[b, r], :] W^T + bias); S = None: every row (the
     dense block). X [B, N, d_in] bf16, Wt [d_out, d_in] bf16, S [B, k] int32,
-    bias [d_out] fp32, act "none" or "gelu_tanh". Returns [B, k or N, d_out]."""
+    bias [d_out] fp32, act "none" or "gelu_tanh". Returns [B, k or N, d_out].
+    ws: the workspace for the compact copy of the rows of S (a fresh one when
+    None; False: the GEMM gathers the rows itself)."""
     _need(X, "X", torch.bfloat16, 3)
     B, N, d_in = X.shape
     dev = X.device
@@ -469,6 +477,12 @@ def gather_linear(X, Wt, S=None, bias=None, act="none", out=None):
     if act not in _ACTS:
         raise ValueError(f"act must be one of {sorted(_ACTS)}, got {act!r}")
     out = _out(out, "out", torch.bfloat16, (B, R, d_out), dev)
+    w, wb = None, 0
+    if S is not None and ws is not False:
+        if ws is None:
+            ws = torch.empty(gather_linear_workspace_bytes(B, k, d_in), dtype=torch.uint8, device=dev)
+        _need(ws, "ws", torch.uint8, 1, device=dev)
+        w, wb = ws, ws.numel()
     _check("safe_gather_linear", lib().safe_gather_linear(_p(X), _p(S), k, _p(Wt), _p(bias), _ACTS[act], _p(out), B,
-                                                          N, d_in, d_out, _stream()))
+                                                          N, d_in, d_out, _p(w), wb, _stream()))
     return out

@@ -61,7 +61,9 @@ class BlockAttention:
       sigma      Eq. (11) smoothing before the split (None: raw scores), on
                  the grid_h x grid_w latent grid
       assembled  SRSU with K/V of S u C assembled in the kernel (no scatter;
-                 the cache is only read between anchors)
+                 the cache is only read between anchors). Off by default: at
+                 the 2560^2 workload this form is measured slower than the
+                 scatter followed by SRSU that the default runs.
     """
 
     def __init__(self, schedule: AnchorSchedule, B: int, N: int, H: int, d: int, k: int, device,

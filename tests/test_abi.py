@@ -47,7 +47,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.safe_abi_version() == 5
+    assert lib.safe_abi_version() == 6
     assert lib.safe_status_string(0) == b"ok"
     assert lib.safe_status_string(1) == b"invalid argument"
     assert lib.safe_status_string(99) == b"unknown status"
@@ -79,6 +79,13 @@ def test_host_validation_rejects_bad_arguments_without_gpu(lib):
     assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 0, 1, 96, 1.0, null, 0, null) == 1
     assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 80, 1.0, null, 0, null) == 2
     assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 96, float("nan"), null, 0, null) == 1
+    # the logit scale must be positive (the kernels scale each row's maximum)
+    for bad in (0.0, -0.1, float("-inf")):
+        assert lib.safe_attn_self(fake, fake, fake, fake, null, 1, 16, 1, 96, bad, null, 0, null) == 1
+        assert lib.safe_srsu_attn(fake, 0, fake, 4, fake, fake, fake, null, 1, 16, 1, 96, bad, null, 0, null) == 1
+        assert lib.safe_attn_cross(fake, null, 16, fake, fake, fake, fake, 1, 16, 16, 1, 96, bad, null) == 1
+        assert lib.safe_pcsp_topk(fake, fake, fake, null, 1, 16, 16, 1, 96, bad, fake, 0, 4, fake, null, fake,
+                                  4096, null) == 1
     # SRSU: k out of range
     assert lib.safe_srsu_attn(fake, 0, fake, 0, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
     assert lib.safe_srsu_attn(fake, 0, fake, 17, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
@@ -91,15 +98,18 @@ def test_host_validation_rejects_bad_arguments_without_gpu(lib):
     assert asm(fake, 0, fake, 17, fake, fake, 1, fake, fake, fake, null, 1, 16, 1, 96, 1.0, null, 0, null) == 1
     assert asm(fake, 0, fake, 4, fake, fake, 1, fake, fake, fake, null, 1, 16, 1, 80, 1.0, null, 0, null) == 2
     # row-wise layer: widths multiples of 8, act 0/1, k in [1, N] with S, aligned bias
+    lib.safe_gather_linear_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.safe_gather_linear_workspace_bytes(2, 6400, 2304) == 2 * 6400 * 2304 * 2
+    assert lib.safe_gather_linear_workspace_bytes(0, 6400, 2304) == 0
     gl = lib.safe_gather_linear
-    assert gl(fake, null, 0, fake, null, 0, fake, 1, 16, 60, 64, null) == 1
-    assert gl(fake, null, 0, fake, null, 0, fake, 1, 16, 56, 64, null) == 1
-    assert gl(fake, null, 0, fake, null, 0, fake, 1, 16, 64, 4, null) == 1
-    assert gl(fake, null, 0, fake, null, 2, fake, 1, 16, 64, 64, null) == 1
-    assert gl(fake, fake, 0, fake, null, 0, fake, 1, 16, 64, 64, null) == 1
-    assert gl(fake, fake, 17, fake, null, 0, fake, 1, 16, 64, 64, null) == 1
-    assert gl(fake, null, 0, fake, ctypes.c_void_p(0x10002), 0, fake, 1, 16, 64, 64, null) == 1
-    assert gl(odd, null, 0, fake, null, 0, fake, 1, 16, 64, 64, null) == 1
+    assert gl(fake, null, 0, fake, null, 0, fake, 1, 16, 60, 64, null, 0, null) == 1
+    assert gl(fake, null, 0, fake, null, 0, fake, 1, 16, 56, 64, null, 0, null) == 1
+    assert gl(fake, null, 0, fake, null, 0, fake, 1, 16, 64, 4, null, 0, null) == 1
+    assert gl(fake, null, 0, fake, null, 2, fake, 1, 16, 64, 64, null, 0, null) == 1
+    assert gl(fake, fake, 0, fake, null, 0, fake, 1, 16, 64, 64, null, 0, null) == 1
+    assert gl(fake, fake, 17, fake, null, 0, fake, 1, 16, 64, 64, null, 0, null) == 1
+    assert gl(fake, null, 0, fake, ctypes.c_void_p(0x10002), 0, fake, 1, 16, 64, 64, null, 0, null) == 1
+    assert gl(odd, null, 0, fake, null, 0, fake, 1, 16, 64, 64, null, 0, null) == 1
     # cross: M > 256 unsupported, nq must equal N without q_idx
     assert lib.safe_attn_cross(fake, null, 16, fake, fake, fake, fake, 1, 16, 257, 1, 96, 1.0, null) == 2
     assert lib.safe_attn_cross(fake, null, 8, fake, fake, fake, fake, 1, 16, 16, 1, 96, 1.0, null) == 1
@@ -180,4 +190,4 @@ def test_graft_entry_build_loads_the_library():
     # checks the ABI version it was written against
     import __graft_entry__ as g
     g.build()
-    assert ops.abi_version() == 5
+    assert ops.abi_version() == 6

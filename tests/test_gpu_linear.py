@@ -58,11 +58,16 @@ def _check(got, Xsel64, Wt64, bias64, act):
     (2, 4096, 128, 1000, 1229, "gelu_tanh", False),
     (2, 8192, 256, 2048, 4096, "gelu_tanh", True),  # 512 tiles: several per CTA, both accumulators
 ])
-def test_gather_linear_parity(B, N, d_in, d_out, k, act, with_bias):
+@pytest.mark.parametrize("compact_copy", [True, False])
+def test_gather_linear_parity(B, N, d_in, d_out, k, act, with_bias, compact_copy):
+    # compact_copy: the rows of S copied into the workspace first (the
+    # default); else gathered by the GEMM itself (no workspace)
+    if k is None and not compact_copy:
+        pytest.skip("every row: no gather either way")
     X, Wt, bias = _layer(B, N, d_in, d_out, seed=N + d_out)
     S = _rows(B, N, k, seed=k) if k is not None else None
     got = ops.gather_linear(X.to(DEV), Wt.to(DEV), None if S is None else torch.from_numpy(S).to(DEV),
-                            None if bias is None else bias.to(DEV), act=act)
+                            None if bias is None else bias.to(DEV), act=act, ws=None if compact_copy else False)
     X64 = to64(X)
     Xsel = X64 if S is None else np.stack([X64[b, S[b]] for b in range(B)])
     _check(got, Xsel, to64(Wt), None if bias is None else bias.numpy().astype(np.float64), act)
@@ -75,14 +80,15 @@ def test_gathered_rows_equal_dense_rows_bitwise():
     Xd, Wd, bd = X.to(DEV), Wt.to(DEV), bias.to(DEV)
     S = torch.from_numpy(_rows(B, N, k, seed=3)).to(DEV)
     dense = ops.gather_linear(Xd, Wd, bias=bd, act="gelu_tanh")
-    sel = ops.gather_linear(Xd, Wd, S=S, bias=bd, act="gelu_tanh")
-    for b in range(B):
-        assert torch.equal(sel[b], dense[b, S[b].long()])
-    # rows in any order, repeated rows included
-    Sr = torch.tensor([[5, 5, 699, 0], [3, 2, 1, 0]], dtype=torch.int32, device=DEV)
-    sel = ops.gather_linear(Xd, Wd, S=Sr, bias=bd, act="gelu_tanh")
-    for b in range(B):
-        assert torch.equal(sel[b], dense[b, Sr[b].long()])
+    for ws in (None, False):  # compact copy first / gathered by the GEMM
+        sel = ops.gather_linear(Xd, Wd, S=S, bias=bd, act="gelu_tanh", ws=ws)
+        for b in range(B):
+            assert torch.equal(sel[b], dense[b, S[b].long()])
+        # rows in any order, repeated rows included
+        Sr = torch.tensor([[5, 5, 699, 0], [3, 2, 1, 0]], dtype=torch.int32, device=DEV)
+        sel = ops.gather_linear(Xd, Wd, S=Sr, bias=bd, act="gelu_tanh", ws=ws)
+        for b in range(B):
+            assert torch.equal(sel[b], dense[b, Sr[b].long()])
     assert ops.device_status() == 0
 
 
@@ -104,8 +110,9 @@ def test_gather_linear_out_of_range_row_flagged_not_faulted():
     X, Wt, _ = _layer(B, N, d_in, d_out, seed=23)
     Xd, Wd = X.to(DEV), Wt.to(DEV)
     S = torch.tensor([[7, 200, -1, 3]], dtype=torch.int32, device=DEV)
-    got = ops.gather_linear(Xd, Wd, S=S)
-    assert ops.device_status() & (1 << ops.SAFE_ERR_DEVICE_CHECK)
     dense = ops.gather_linear(Xd, Wd)
-    assert torch.equal(got[0, 0], dense[0, 7]) and torch.equal(got[0, 3], dense[0, 3])
-    assert torch.equal(got[0, 1], dense[0, 0]) and torch.equal(got[0, 2], dense[0, 0])  # replaced by row 0
+    for ws in (None, False):  # compact copy first / gathered by the GEMM
+        got = ops.gather_linear(Xd, Wd, S=S, ws=ws)
+        assert ops.device_status() & (1 << ops.SAFE_ERR_DEVICE_CHECK)
+        assert torch.equal(got[0, 0], dense[0, 7]) and torch.equal(got[0, 3], dense[0, 3])
+        assert torch.equal(got[0, 1], dense[0, 0]) and torch.equal(got[0, 2], dense[0, 0])  # replaced by row 0

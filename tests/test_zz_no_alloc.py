@@ -7,8 +7,10 @@ collected last on purpose, so a run that stops at the first failure has
 already run every other test; it also passes on its own in a fresh process.
 
 Checked through the C ABI against safe_pcsp_topk (the workspace entry point)
-on two calls in a row, within the PCSP score tolerance of the other tests,
-plus the size limit.
+on two calls in a row: both run the same kernels on the same inputs, only
+the scratch address differs, so scores, S and C must be bit-identical. The
+scores are also compared with the fp64 oracle at the PCSP score tolerance of
+the other tests, and the size limit is checked.
 """
 
 import ctypes
@@ -18,6 +20,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from mask_free_b200 import ops, synth
 
 pytestmark = pytest.mark.gpu
@@ -42,6 +45,7 @@ def test_noalloc_pcsp_matches_workspace_entry_point_on_two_calls():
     lens = lens.to(DEV)
     scores_new = torch.zeros((B, N), dtype=torch.float32, device=DEV)
     scores_ref = torch.zeros_like(scores_new)
+    ref = np.zeros((B, N))
     for call in range(2):
         Q = synth.normal_bf16((B, N, H, d), 900 + call).to(DEV)
         Ky = synth.normal_bf16((B, M, H, d), 910 + call).to(DEV)
@@ -52,10 +56,12 @@ def test_noalloc_pcsp_matches_workspace_entry_point_on_two_calls():
         assert st == ops.SAFE_OK
         _, S_ref, C_ref = ops.pcsp_topk(Q, Ky, lens, w, scores=scores_ref, accumulate=bool(accumulate), k=k)
         torch.cuda.synchronize()
-        np.testing.assert_allclose(scores_new.cpu().numpy(), scores_ref.cpu().numpy(), rtol=2e-5, atol=1e-8)
-        if torch.equal(scores_new, scores_ref):
-            assert torch.equal(S_new, S_ref) and torch.equal(C_new, C_ref)
+        assert torch.equal(scores_new, scores_ref), f"call {call}: scores differ from the workspace entry point"
+        assert torch.equal(S_new, S_ref) and torch.equal(C_new, C_ref), f"call {call}: partition differs"
         assert ops.device_status() == 0
+        ref = ref + O.pcsp_scores(synth.bf16_to_f64(Q.cpu()), synth.bf16_to_f64(Ky.cpu()), lens.cpu().numpy(),
+                                  w.cpu().numpy(), 1.0 / math.sqrt(d))
+        np.testing.assert_allclose(scores_new.cpu().numpy(), ref, rtol=3e-5, atol=1e-8)
 
 
 def test_noalloc_pcsp_rejects_sizes_beyond_the_scratch():
