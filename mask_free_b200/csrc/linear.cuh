@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3, row = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0;
     for (int i = 0; i < n_local; ++i) {
       const int a = i & 1;
       if (!warp_wait(&acc_full[a], (i >> 1) & 1, &abort_flag)) break;
@@ -232,14 +233,30 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
         }
         const int nc = n0 + 32 * c;
         if (nc >= p.d_out) continue;
+        // the chunk's 32 bias values: 8 vector loads (the same for every
+        // row, so they come from L1), or element by element at the ragged
+        // last chunk or a bias that is not 16-byte aligned
+        float bv[32];
+        if (p.bias == nullptr) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) bv[e] = 0.f;
+        } else if (bias_vec && nc + 32 <= p.d_out) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + nc) + u);
+            bv[4 * u] = b4.x;
+            bv[4 * u + 1] = b4.y;
+            bv[4 * u + 2] = b4.z;
+            bv[4 * u + 3] = b4.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) bv[e] = nc + e < p.d_out ? __ldg(p.bias + nc + e) : 0.f;
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float f0 = __uint_as_float(v[2 * e]), f1 = __uint_as_float(v[2 * e + 1]);
-          if (p.bias != nullptr) {
-            f0 += nc + 2 * e < p.d_out ? __ldg(p.bias + nc + 2 * e) : 0.f;
-            f1 += nc + 2 * e + 1 < p.d_out ? __ldg(p.bias + nc + 2 * e + 1) : 0.f;
-          }
+          float f0 = __uint_as_float(v[2 * e]) + bv[2 * e], f1 = __uint_as_float(v[2 * e + 1]) + bv[2 * e + 1];
           if (p.act == 1) {
             f0 = gelu_tanh_f(f0);
             f1 = gelu_tanh_f(f1);

@@ -392,28 +392,4 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair on the FMA pipe (Cody-Waite split x = n + f with n the
-// nearest integer, then a degree-3 minimax polynomial for 2^f on
-// [-1/2, 1/2] fitted by iteratively reweighted least squares; max relative
-// error 8.4e-5, far below the bf16 rounding of the probabilities). x is
-// clamped to >= -126 so the exponent add cannot wrap; results below 2^-126
-// are negligible next to the row sum.
-__device__ __forceinline__ uint64_t exp2_poly_f2(float x0, float x1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
-  const uint64_t r = f2_add(t, f2_pack(-kShift, -kShift));                       // round(x)
-  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);                          // x - round(x)
-  uint64_t p = f2_fma(f2_pack(0.055213045f, 0.055213045f), f, f2_pack(0.24271424f, 0.24271424f));
-  p = f2_fma(p, f, f2_pack(0.69326216f, 0.69326216f));
-  p = f2_fma(p, f, f2_pack(0.99991959f, 0.99991959f));
-  // scale by 2^n: add n to the exponent field (t's low mantissa bits hold n)
-  const uint32_t t0 = static_cast<uint32_t>(t), t1 = static_cast<uint32_t>(t >> 32);
-  const uint32_t p0 = static_cast<uint32_t>(p), p1 = static_cast<uint32_t>(p >> 32);
-  const uint32_t e0 = p0 + (t0 << 23), e1 = p1 + (t1 << 23);
-  return (static_cast<uint64_t>(e1) << 32) | e0;
-}
-
 }  // namespace safe
