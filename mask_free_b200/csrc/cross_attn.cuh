@@ -450,37 +450,62 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         }
         if (!ok) return false;
       } else {
-        // (aliased layout only) pass 1: row max over valid keys (the key
-        // tests are redundant with the -inf columns but keep this path's
-        // registers low)
-        float mx = -INFINITY;
-        for (int c = 0; c < Lp / 32; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tS + 32 * c, sr);
-          tmem_ld_wait32(sr);
+        // (aliased layout only) two passes over S, 32 keys at a time,
+        // specialised on the number NC of chunks: pass 1 the row max, pass 2
+        // the probabilities, the sums and P (P chunk c lands on S columns
+        // already read). The padding columns hold -inf from the mask step of
+        // the S product and weight 0, so no key needs a test.
+        auto two_pass = [&](auto nc_tag) {
+          constexpr int NC = decltype(nc_tag)::value;
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i2 = 0; i2 < 32; ++i2)
-            if (32 * c + i2 < L) mx = fmaxf(mx, __uint_as_float(sr[i2]));
-        }
-        const float neg = -mx * sl2;
-        // pass 2: probabilities, sums, P -> TMEM (P chunk c lands on S
-        // columns already read)
-        for (int c = 0; c < Lp / 32; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tS + 32 * c, sr);
-          tmem_ld_wait32(sr);
-          uint32_t pk[16];
+          for (int c = 0; c < NC; ++c) {
+            uint32_t sr[32];
+            tmem_ld32(tS + 32 * c, sr);
+            tmem_ld_wait32(sr);
 #pragma unroll
-          for (int i2 = 0; i2 < 16; ++i2) {
-            const int j0 = 32 * c + 2 * i2;
-            const float a = j0 < L ? ex2_approx(fmaf(__uint_as_float(sr[2 * i2]), sl2, neg)) : 0.f;
-            const float bb = j0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(sr[2 * i2 + 1]), sl2, neg)) : 0.f;
-            l += a + bb;
-            score = fmaf(sw[j0], a, score);
-            score = fmaf(sw[j0 + 1], bb, score);
-            pk[i2] = pack_bf16x2(a, bb);
+            for (int j = 0; j < 32; j += 8)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                m4[q] = fmax3(m4[q], __uint_as_float(sr[j + 2 * q]), __uint_as_float(sr[j + 2 * q + 1]));
           }
-          if (has_o) tmem_st16(tP + 16 * c, pk);
+          const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+          const uint64_t sl2x2 = f2_pack(sl2, sl2), neg2 = f2_pack(-mx * sl2, -mx * sl2);
+          uint64_t lacc[2] = {0, 0}, sacc[2] = {0, 0};  // packed row sums and weighted sums
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
+            uint32_t sr[32];
+            tmem_ld32(tS + 32 * c, sr);
+            tmem_ld_wait32(sr);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i2 = 0; i2 < 16; ++i2) {
+              const int j0 = 32 * c + 2 * i2;
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i2]), __uint_as_float(sr[2 * i2 + 1])), sl2x2, neg2),
+                        x0, x1);
+              const float a = ex2_approx(x0), bb = ex2_approx(x1);
+              const uint64_t e2 = f2_pack(a, bb);
+              const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
+              lacc[i2 & 1] = f2_add(lacc[i2 & 1], e2);
+              sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+              pk[i2] = pack_bf16x2(a, bb);
+            }
+            if (has_o) tmem_st16(tP + 16 * c, pk);
+          }
+          float l0, l1, l2, l3, s0, s1, s2, s3;
+          f2_unpack(lacc[0], l0, l1);
+          f2_unpack(lacc[1], l2, l3);
+          f2_unpack(sacc[0], s0, s1);
+          f2_unpack(sacc[1], s2, s3);
+          l = (l0 + l1) + (l2 + l3);
+          score = (s0 + s1) + (s2 + s3);
+        };
+        switch (Lp / 32) {
+          case 5: two_pass(std::integral_constant<int, 5>{}); break;
+          case 6: two_pass(std::integral_constant<int, 6>{}); break;
+          case 7: two_pass(std::integral_constant<int, 7>{}); break;
+          default: two_pass(std::integral_constant<int, 8>{}); break;
         }
         if (!has_o) {
           tc_fence_before();
