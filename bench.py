@@ -181,14 +181,14 @@ class Step:
         self.ws = torch.empty(ops.pcsp_workspace_bytes(B, N, H), dtype=torch.uint8, device=dev)
         self.cls = torch.empty(3, dtype=torch.int64, device=dev)
         self.ws_self = torch.empty(max(256, ops.attn_workspace_bytes(B, N, N, H, d)), dtype=torch.uint8, device=dev)
-        self.ws_srsu = torch.empty(max(256, ops.attn_workspace_bytes(B, k, N, H, d)), dtype=torch.uint8, device=dev)
+        self.ws_srsu = torch.empty(max(256, ops.srsu_workspace_bytes(B, k, N, H, d)), dtype=torch.uint8, device=dev)
         self.Kc, self.Vc = inp["Kc"].clone(), inp["Vc"].clone()
         self.events = []
         # library kernels per step: classify 3 (init, rows, verdict); dense 1
         # (+1 merge when the last wave is split along the keys); cross with
-        # PCSP 3 (cross, head sum, top-k); scatter 1; SRSU 1 (+1 merge);
-        # cross on S 1
-        self.launches = 3 + 1 + (ops.attn_workspace_bytes(B, N, N, H, d) > 0) + 3 + 1 + 1 + \
+        # PCSP 3 (cross, head sum, top-k); scatter 1; SRSU 2 (query-row copy,
+        # attention; +1 merge); cross on S 1
+        self.launches = 3 + 1 + (ops.attn_workspace_bytes(B, N, N, H, d) > 0) + 3 + 1 + 2 + \
             (ops.attn_workspace_bytes(B, k, N, H, d) > 0) + 1
 
     def __call__(self, timed=False):
@@ -269,7 +269,7 @@ def kernel_table(dev, pk):
         Os = torch.empty((s.B, k, s.H, s.d), dtype=torch.bfloat16, device=dev)
         dense_f, srsu_f, cross_f, _ = flops(s, lsum, k)
         ws_d = torch.empty(max(256, ops.attn_workspace_bytes(s.B, s.N, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
-        ws_s = torch.empty(max(256, ops.attn_workspace_bytes(s.B, k, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
+        ws_s = torch.empty(max(256, ops.srsu_workspace_bytes(s.B, k, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
         t_d = time_kernel(lambda: ops.attn_self(inp["Q"], inp["K"], inp["V"], out=O, ws=ws_d))
         t_s = time_kernel(lambda: ops.srsu_attn(inp["Q"], S, inp["Kc"], inp["Vc"], out=Os, ws=ws_s))
         Ox = torch.empty_like(O)
@@ -381,7 +381,7 @@ def kernel_table(dev, pk):
                 kk = max(1, math.ceil(rho * s.N))
                 Sr = torch.sort(torch.randperm(s.N, device=dev)[:kk])[0].to(torch.int32).expand(s.B, kk).contiguous()
                 Osr = torch.empty((s.B, kk, s.H, s.d), dtype=torch.bfloat16, device=dev)
-                wsr = torch.empty(max(256, ops.attn_workspace_bytes(s.B, kk, s.N, s.H, s.d)), dtype=torch.uint8,
+                wsr = torch.empty(max(256, ops.srsu_workspace_bytes(s.B, kk, s.N, s.H, s.d)), dtype=torch.uint8,
                                   device=dev)
                 sweep[str(rho)] = time_kernel(lambda: ops.srsu_attn(inp["Q"], Sr, inp["Kc"], inp["Vc"], out=Osr,
                                                                     ws=wsr), reps=10)
@@ -412,7 +412,7 @@ def sequence_n36864(dev, pk):
     Osx = torch.empty_like(Os)
     dense_f, srsu_f, cross_f, cross_s_f = flops(s, lsum, k)
     ws_d = torch.empty(max(256, ops.attn_workspace_bytes(s.B, s.N, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
-    ws_s = torch.empty(max(256, ops.attn_workspace_bytes(s.B, k, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(max(256, ops.srsu_workspace_bytes(s.B, k, s.N, s.H, s.d)), dtype=torch.uint8, device=dev)
     Kc, Vc = inp["Kc"], inp["Vc"]
     t_d = time_kernel(lambda: ops.attn_self(inp["Q"], inp["K"], inp["V"], out=O, ws=ws_d), reps=5)
     t_s = time_kernel(lambda: ops.srsu_attn(inp["Q"], S, Kc, Vc, out=Os, ws=ws_s), reps=10)

@@ -56,7 +56,7 @@ typedef enum {
 
 typedef enum { SAFE_BOOL = 0, SAFE_U8 = 1, SAFE_F32 = 2, SAFE_F16 = 3, SAFE_BF16 = 4 } safe_dtype;
 
-/* ABI version of this header (bumped on any signature or entry-point change): 6. */
+/* ABI version of this header (bumped on any signature or entry-point change): 7. */
 int safe_abi_version(void);
 const char* safe_status_string(int status);
 
@@ -216,8 +216,16 @@ safe_status safe_topk_partition(const float* scores, int B, int N, int k, int32_
  *  S        device int32 [B, k], strictly ascending, values in [0, N).
  *  Kc, Vc   device bf16 [B, N, H, d].
  *  O_S      device bf16 [B, k, H, d] (written); lse device fp32 [B, H, k] or NULL.
- *  ws       as safe_attn_self, sized safe_attn_workspace_bytes(B, k, N, H, d).
+ *  ws       device workspace (16-byte aligned, caller-owned, contents
+ *           undefined after the call) of ws_bytes bytes, or NULL:
+ *           safe_srsu_workspace_bytes(B, k, N, H, d) bytes: with
+ *           q_compact = 0 the rows of S are first copied out of Q into it as a
+ *           compact [B, k, H, d] tensor (faster than gathering them inside
+ *           the attention kernel), and the rest serves the key split;
+ *           safe_attn_workspace_bytes(B, k, N, H, d) bytes: the key split
+ *           only; less: neither (every result is the same bit for bit).
  */
+size_t safe_srsu_workspace_bytes(int B, int k, int N, int H, int d);
 safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
                            void* O_S, float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
                            void* stream);

@@ -23,7 +23,7 @@ using namespace safe;
 
 namespace {
 
-constexpr int kAbiVersion = 6;
+constexpr int kAbiVersion = 7;
 constexpr float kLog2e = 1.4426950408889634f;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -361,6 +361,31 @@ bool fill_srsu(FlashParams& p, const void* Q, int q_compact, const int32_t* S, i
   return true;
 }
 
+// With the query rows gathered from a full-size Q and room for them in the
+// workspace (safe_srsu_workspace_bytes): copy the rows of S into the end of
+// the workspace as a compact [B, k, H, d] tensor and point Q there, so the
+// kernel loads each query tile by one tiled copy instead of per-row gathers;
+// the rest of the workspace is left for the key split. False on a launch
+// error.
+bool srsu_compact_q(const void*& Q, int& q_compact, const int32_t* S, int k, int B, int N, int H, int d, void* ws,
+                    size_t& ws_bytes, cudaStream_t s) {
+  if (q_compact || ws == nullptr || !aligned16(ws)) return true;
+  const size_t split = align256(safe_attn_workspace_bytes(B, k, N, H, d));
+  const size_t need = split + static_cast<size_t>(B) * k * H * d * 2;
+  if (ws_bytes < need) return true;
+  const long long rows = static_cast<long long>(B) * k;
+  if ((rows + 7) / 8 > INT_MAX) return true;
+  void* qc = static_cast<uint8_t*>(ws) + split;
+  gather_rows_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(static_cast<const uint4*>(Q), S,
+                                                                           static_cast<uint4*>(qc), B, N, k,
+                                                                           H * d / 8);
+  if (cudaGetLastError() != cudaSuccess) return false;
+  Q = qc;
+  q_compact = 1;
+  ws_bytes = split;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -454,6 +479,11 @@ safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O,
   return dispatch_flash(d, p, ws, ws_bytes, as_stream(stream));
 }
 
+size_t safe_srsu_workspace_bytes(int B, int k, int N, int H, int d) {
+  if (B < 1 || k < 1 || N < 1 || H < 1 || !supported_d(d)) return 0;
+  return align256(safe_attn_workspace_bytes(B, k, N, H, d)) + static_cast<size_t>(B) * k * H * d * 2;
+}
+
 safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k, const void* Kc, const void* Vc,
                            void* O_S, float* lse, int B, int N, int H, int d, float scale, void* ws, size_t ws_bytes,
                            void* stream) {
@@ -461,6 +491,7 @@ safe_status safe_srsu_attn(const void* Q, int q_compact, const int32_t* S, int k
   if (!sizes_ok(B, N, H) || k < 1 || k > N || !scale_ok(scale)) return SAFE_ERR_INVALID_ARG;
   if (!q_compact && S == nullptr) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
+  if (!srsu_compact_q(Q, q_compact, S, k, B, N, H, d, ws, ws_bytes, as_stream(stream))) return SAFE_ERR_CUDA;
   FlashParams p{};
   if (!fill_srsu(p, Q, q_compact, S, k, Kc, Vc, O_S, lse, B, N, H, d, scale)) return SAFE_ERR_CUDA;
   return dispatch_flash(d, p, ws, ws_bytes, as_stream(stream));
@@ -475,6 +506,7 @@ safe_status safe_srsu_attn_assembled(const void* Q, int q_compact, const int32_t
     return SAFE_ERR_INVALID_ARG;
   if (!sizes_ok(B, N, H) || k < 1 || k > N || !scale_ok(scale)) return SAFE_ERR_INVALID_ARG;
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
+  if (!srsu_compact_q(Q, q_compact, S, k, B, N, H, d, ws, ws_bytes, as_stream(stream))) return SAFE_ERR_CUDA;
   FlashParams p{};
   if (!fill_srsu(p, Q, q_compact, S, k, Kc, Vc, O_S, lse, B, N, H, d, scale)) return SAFE_ERR_CUDA;
   p.k_cur = static_cast<const __nv_bfloat16*>(Kcur);

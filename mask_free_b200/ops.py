@@ -35,6 +35,7 @@ _SIGS = {
     "safe_pcsp_workspace_bytes": [_i, _i, _i],
     "safe_pcsp_topk": [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp],
     "safe_topk_partition": [_vp, _i, _i, _i, _vp, _vp, _vp],
+    "safe_srsu_workspace_bytes": [_i, _i, _i, _i, _i],
     "safe_srsu_attn": [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp],
     "safe_srsu_attn_assembled": [_vp, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz,
                                  _vp],
@@ -53,7 +54,7 @@ _SIGS = {
     "safe_gather_linear": [_vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _sz, _vp],
 }
 _RESTYPES = {"safe_pcsp_workspace_bytes": _sz, "safe_attn_workspace_bytes": _sz, "safe_sensitivity_workspace_bytes": _sz,
-             "safe_gather_linear_workspace_bytes": _sz,
+             "safe_gather_linear_workspace_bytes": _sz, "safe_srsu_workspace_bytes": _sz,
              "safe_status_string": ctypes.c_char_p}
 
 
@@ -305,6 +306,24 @@ def topk_partition(scores, k, S=None, C=None, with_c=True):
     return S, C
 
 
+def srsu_workspace_bytes(B: int, k: int, N: int, H: int, d: int) -> int:
+    return int(lib().safe_srsu_workspace_bytes(B, k, N, H, d))
+
+
+def _srsu_ws(ws, B, k, N, H, d, device):
+    """Workspace of an SRSU call: the given tensor, a fresh one of
+    srsu_workspace_bytes (ws=None: room for the compact query rows and the
+    key split), or none (ws=False)."""
+    if ws is False:
+        return None, 0
+    if ws is None:
+        nbytes = srsu_workspace_bytes(B, k, N, H, d)
+        if nbytes == 0:
+            return None, 0
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
 def _srsu_args(Q, S, Kc, Vc, q_compact):
     """Check the SRSU inputs: cache K/V [B, N, H, d], S [B, k], Q [B, k, H, d]
     (compact) or [B, N, H, d]; returns B, N, H, d, k, device."""
@@ -326,7 +345,7 @@ def srsu_attn(Q, S, Kc, Vc, q_compact=False, scale=None, return_lse=False, out=N
     out = _out(out, "out", torch.bfloat16, (B, k, H, d), dev)
     if return_lse:
         lse = _out(lse, "lse", torch.float32, (B, H, k), dev)
-    w, wb = _attn_ws(ws, B, k, N, H, d, dev)
+    w, wb = _srsu_ws(ws, B, k, N, H, d, dev)
     _check("safe_srsu_attn", lib().safe_srsu_attn(_p(Q), 1 if q_compact else 0, _p(S), k, _p(Kc), _p(Vc), _p(out),
                                                   _p(lse if return_lse else None), B, N, H, d, _scale(d, scale),
                                                   _p(w), wb, _stream()))
@@ -346,7 +365,7 @@ def srsu_attn_assembled(Q, S, Kcur, Vcur, Kc, Vc, q_compact=False, cur_compact=F
     out = _out(out, "out", torch.bfloat16, (B, k, H, d), dev)
     if return_lse:
         lse = _out(lse, "lse", torch.float32, (B, H, k), dev)
-    w, wb = _attn_ws(ws, B, k, N, H, d, dev)
+    w, wb = _srsu_ws(ws, B, k, N, H, d, dev)
     _check("safe_srsu_attn_assembled", lib().safe_srsu_attn_assembled(
         _p(Q), 1 if q_compact else 0, _p(S), k, _p(Kcur), _p(Vcur), 1 if cur_compact else 0, _p(Kc), _p(Vc), _p(out),
         _p(lse if return_lse else None), B, N, H, d, _scale(d, scale), _p(w), wb, _stream()))

@@ -47,7 +47,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.safe_abi_version() == 6
+    assert lib.safe_abi_version() == 7
     assert lib.safe_status_string(0) == b"ok"
     assert lib.safe_status_string(1) == b"invalid argument"
     assert lib.safe_status_string(99) == b"unknown status"
@@ -59,6 +59,12 @@ def test_attn_workspace_plan(lib):
     lib.safe_attn_workspace_bytes.restype = ctypes.c_size_t
     assert lib.safe_attn_workspace_bytes(2, 6400, 25600, 24, 96) > 0      # 1200 units: 8.1 waves
     assert lib.safe_attn_workspace_bytes(1, 256, 256, 2, 64) == 0         # 2 key tiles: no split
+    # SRSU: the key split's workspace (256-byte aligned) plus the compact query rows
+    lib.safe_srsu_workspace_bytes.restype = ctypes.c_size_t
+    split = lib.safe_attn_workspace_bytes(2, 6400, 25600, 24, 96)
+    assert lib.safe_srsu_workspace_bytes(2, 6400, 25600, 24, 96) == ((split + 255) // 256) * 256 + 2 * 6400 * 24 * 96 * 2
+    assert lib.safe_srsu_workspace_bytes(1, 64, 256, 2, 64) == 64 * 2 * 64 * 2
+    assert lib.safe_srsu_workspace_bytes(1, 64, 256, 2, 80) == 0
     assert lib.safe_attn_workspace_bytes(0, 256, 256, 2, 64) == 0
     assert lib.safe_attn_workspace_bytes(1, 256, 256, 2, 80) == 0
 
@@ -190,4 +196,4 @@ def test_graft_entry_build_loads_the_library():
     # checks the ABI version it was written against
     import __graft_entry__ as g
     g.build()
-    assert ops.abi_version() == 6
+    assert ops.abi_version() == 7

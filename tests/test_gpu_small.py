@@ -464,6 +464,33 @@ def test_key_split_wave_balancing_matches_oracle(B, N, H, d, k):
     assert ops.device_status() == 0
 
 
+@pytest.mark.parametrize("B,N,H,d,k", [(2, 4096, 3, 96, 1229), (1, 1000, 2, 64, 333), (2, 700, 2, 128, 700)])
+def test_srsu_compact_query_copy_is_bit_identical(B, N, H, d, k):
+    # with room for the compact query rows the entry point copies the rows of
+    # S out of Q first and loads compact tiles; the attention-only workspace
+    # and no workspace gather them in the kernel: the same bits either way,
+    # and the same as a caller-compacted Q
+    Q, K, V = rand_qkv(B, N, H, d, seed=2 * N + k)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    S = np.stack([np.sort(np.random.default_rng(b + 11).choice(N, k, replace=False)) for b in range(B)])
+    Sd = torch.from_numpy(S.astype(np.int32)).to(DEV)
+    full = ops.srsu_workspace_bytes(B, k, N, H, d)
+    split = ops.attn_workspace_bytes(B, k, N, H, d)
+    assert full >= split + B * k * H * d * 2
+    ws = torch.full((full // 4,), float("nan"), dtype=torch.float32, device=DEV).view(torch.uint8)
+    out_copy = ops.srsu_attn(Qd, Sd, Kd, Vd, ws=ws)
+    out_gather = ops.srsu_attn(Qd, Sd, Kd, Vd, ws=ws[:max(split, 1)] if split else False)
+    out_none = ops.srsu_attn(Qd, Sd, Kd, Vd, ws=False)
+    Qc = torch.stack([Qd[b, Sd[b].long()] for b in range(B)]).contiguous()
+    out_caller = ops.srsu_attn(Qc, Sd, Kd, Vd, q_compact=True, ws=ws)
+    assert torch.equal(out_copy, out_gather) and torch.equal(out_copy, out_caller)
+    if split == 0:
+        assert torch.equal(out_copy, out_none)
+    ref = O.attention(to64(Q), to64(K), to64(V), 1 / math.sqrt(d), q_rows=S)
+    assert_attn_close(out_copy, ref, "srsu, compact query copy")
+    assert ops.device_status() == 0
+
+
 # ---------------------------------------------------------------- failure detection
 
 
