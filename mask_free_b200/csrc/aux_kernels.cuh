@@ -234,30 +234,68 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot) {
   return res;
 }
 
+// Keys of a sample held in shared memory when N is at most this (160 KB of
+// keys beside the 32 KB of histograms); larger N read them from global
+// memory on every pass.
+constexpr int kTopkSmemKeys = 40960;
+static_assert(kTopkSmemKeys <= 64 * kTopkThreads, "a thread's segment must fit a 64-bit selection mask");
+
 // One CTA per sample b: radix select of the k-th largest key T (8 bits per
 // pass, most significant first), then an ordered compaction: i is selected
 // iff key_i > T, or key_i == T and fewer than r earlier indices had key T
 // (r = k - #{key > T}); selected indices go to S, the rest to C, both in
-// ascending index order.
+// ascending index order. kSmem: the first pass converts the scores once into
+// shared memory (loads batched ahead of the histogram updates); the later
+// passes and the compaction read the keys from there.
+template <bool kSmem>
 __global__ void __launch_bounds__(kTopkThreads) topk_partition_kernel(const float* __restrict__ scores, int N, int k,
                                                                       int32_t* __restrict__ S,
                                                                       int32_t* __restrict__ C) {
+  constexpr int kBatch = 8;
+  extern __shared__ uint32_t topk_keys[];  // [N] when kSmem
   __shared__ int hist[32][256];
   __shared__ int warp_tot[32];
   __shared__ uint32_t sh_prefix;
   __shared__ int sh_remaining;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int b = blockIdx.x;
   const float* sc = scores + static_cast<size_t>(b) * N;
+  auto key_at = [&](int i) -> uint32_t {
+    if constexpr (kSmem)
+      return topk_keys[i];
+    else
+      return score_key(__ldg(sc + i));
+  };
 
   uint32_t prefix = 0, mask = 0;
   int remaining = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int e = tid; e < 32 * 256; e += kTopkThreads) (&hist[0][0])[e] = 0;
     __syncthreads();
-    for (int i = tid; i < N; i += kTopkThreads) {
-      const uint32_t key = score_key(__ldg(sc + i));
-      if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 255u], 1);
+    if (!kSmem || shift == 24) {
+      // global scores: kBatch loads in flight before their histogram updates
+      for (int base = 0; base < N; base += kBatch * kTopkThreads) {
+        float v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int i = base + u * kTopkThreads + tid;
+          v[u] = i < N ? __ldg(sc + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int i = base + u * kTopkThreads + tid;
+          if (i < N) {
+            const uint32_t key = score_key(v[u]);
+            if constexpr (kSmem) topk_keys[i] = key;
+            if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 255u], 1);
+          }
+        }
+      }
+    } else {
+      for (int i = tid; i < N; i += kTopkThreads) {
+        const uint32_t key = topk_keys[i];
+        if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 255u], 1);
+      }
     }
     __syncthreads();
     // count of digit d = 255 - tid; an exclusive scan over the digits from
@@ -283,11 +321,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_partition_kernel(const floa
   const uint32_t T = prefix;
   const int r = remaining;  // keys equal to T that are selected (lowest indices first)
 
+  // each thread a contiguous segment of indices
   const int seg = (N + kTopkThreads - 1) / kTopkThreads;
   const int i0 = min(N, tid * seg), i1 = min(N, i0 + seg);
   int cnt_gt = 0, cnt_eq = 0;
   for (int i = i0; i < i1; ++i) {
-    const uint32_t key = score_key(__ldg(sc + i));
+    const uint32_t key = key_at(i);
     cnt_gt += key > T;
     cnt_eq += key == T;
   }
@@ -297,8 +336,36 @@ __global__ void __launch_bounds__(kTopkThreads) topk_partition_kernel(const floa
   int s_pos = sel_base, c_pos = i0 - sel_base, eq_seen = eq_base;
   int32_t* Sb = S + static_cast<size_t>(b) * k;
   int32_t* Cb = C != nullptr ? C + static_cast<size_t>(b) * (N - k) : nullptr;
+  if constexpr (kSmem) {
+    // the selection as a bit mask over this thread's segment (at most 40
+    // indices), then the key buffer takes the output order: S in [0, k), C
+    // in [k, N); both leave by coalesced stores
+    uint64_t sel_mask = 0;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t key = topk_keys[i];
+      bool sel = key > T;
+      if (key == T) {
+        sel = eq_seen < r;
+        ++eq_seen;
+      }
+      if (sel) sel_mask |= 1ull << (i - i0);
+    }
+    __syncthreads();  // every key has been read
+    c_pos += k;
+    for (int i = i0; i < i1; ++i) {
+      if ((sel_mask >> (i - i0)) & 1ull)
+        topk_keys[s_pos++] = static_cast<uint32_t>(i);
+      else
+        topk_keys[c_pos++] = static_cast<uint32_t>(i);
+    }
+    __syncthreads();
+    for (int e = tid; e < k; e += kTopkThreads) Sb[e] = static_cast<int32_t>(topk_keys[e]);
+    if (Cb != nullptr)
+      for (int e = tid; e < N - k; e += kTopkThreads) Cb[e] = static_cast<int32_t>(topk_keys[k + e]);
+    return;
+  }
   for (int i = i0; i < i1; ++i) {
-    const uint32_t key = score_key(__ldg(sc + i));
+    const uint32_t key = key_at(i);
     bool sel = key > T;
     if (key == T) {
       sel = eq_seen < r;
@@ -310,7 +377,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_partition_kernel(const floa
       Cb[c_pos++] = i;
     }
   }
-  (void)lane;
 }
 
 // ============================================================== wait self-test

@@ -536,7 +536,18 @@ size_t safe_pcsp_workspace_bytes(int B, int N, int H) {
 
 safe_status safe_topk_partition(const float* scores, int B, int N, int k, int32_t* S, int32_t* C, void* stream) {
   if (scores == nullptr || S == nullptr || B < 1 || N < 1 || k < 1 || k > N) return SAFE_ERR_INVALID_ARG;
-  topk_partition_kernel<<<B, kTopkThreads, 0, as_stream(stream)>>>(scores, N, k, S, C);
+  if (N <= kTopkSmemKeys) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+      attr_err = cudaFuncSetAttribute(topk_partition_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kTopkSmemKeys * static_cast<int>(sizeof(uint32_t)));
+    });
+    if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
+    topk_partition_kernel<true><<<B, kTopkThreads, N * sizeof(uint32_t), as_stream(stream)>>>(scores, N, k, S, C);
+  } else {
+    topk_partition_kernel<false><<<B, kTopkThreads, 0, as_stream(stream)>>>(scores, N, k, S, C);
+  }
   return launch_status();
 }
 

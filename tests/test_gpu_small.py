@@ -325,8 +325,11 @@ def test_pcsp_topk_pipeline_valid_against_oracle_scores():
 
 @pytest.mark.parametrize("B,N,k,kind", [(2, 4096, 1229, "normal"), (3, 1000, 1, "ties"), (1, 777, 777, "normal"),
                                         (2, 36864, 7373, "ties"), (1, 1, 1, "normal"), (2, 2049, 1024, "zeros"),
-                                        (1, 5000, 2500, "signed_zero"), (2, 25600, 6400, "few_values")])
+                                        (1, 5000, 2500, "signed_zero"), (2, 25600, 6400, "few_values"),
+                                        (1, 40960, 10240, "normal"), (2, 40961, 9999, "ties"),
+                                        (1, 65536, 16384, "few_values")])
 def test_topk_partition_bit_exact(B, N, k, kind):
+    """Keys in shared memory up to N = 40960, read from global memory above."""
     rng = np.random.default_rng(N + k)
     if kind == "normal":
         s = rng.standard_normal((B, N)).astype(np.float32)
