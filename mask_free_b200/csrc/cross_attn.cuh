@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
     const uint32_t tP = tbase + col_P(g) + lane_addr;
     const float sl2 = p.scale_log2;
     float linv_even = 1.f, linv_odd = 1.f;  // 1 / l of this warpgroup's last two tiles
+    const bool want_score = p.partial != nullptr;
 
     // softmax of tile i: probabilities, l and the PCSP partial; P -> TMEM
     auto softmax = [&](int i) -> bool {
@@ -389,9 +390,11 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
       float l = 0.f, score = 0.f;
       // all of S in registers: one TMEM pass (padding keys hold -inf and
       // weight 0), specialised on the number NC of 32-key chunks so that
-      // every register index is static
-      auto one_pass = [&](auto nc_tag) -> bool {
+      // every register index is static, and on whether the weighted sum of
+      // the PCSP partial is wanted (SC)
+      auto one_pass = [&](auto nc_tag, auto sc_tag) -> bool {
         constexpr int NC = decltype(nc_tag)::value;
+        constexpr bool SC = decltype(sc_tag)::value;
         uint32_t sr[32 * NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) tmem_ld32(tS + 32 * c, sr + 32 * c);
@@ -417,9 +420,11 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), sl2x2, neg2), x0, x1);
           const float a = ex2_approx(x0), bb = ex2_approx(x1);
           const uint64_t e2 = f2_pack(a, bb);
-          const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
           lacc[i2 & 1] = f2_add(lacc[i2 & 1], e2);
-          sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+          if constexpr (SC) {
+            const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
+            sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+          }
           pk[i2] = pack_bf16x2(a, bb);
           if (!kSep && has_o && (i2 & 15) == 15) tmem_st16(tP + (i2 - 15), pk + (i2 - 15));
         }
@@ -442,11 +447,17 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
       };
       if (Lp <= 128) {
         bool ok;
+        const std::true_type sc_on;
+        const std::false_type sc_off;
         switch (Lp / 32) {
-          case 1: ok = one_pass(std::integral_constant<int, 1>{}); break;
-          case 2: ok = one_pass(std::integral_constant<int, 2>{}); break;
-          case 3: ok = one_pass(std::integral_constant<int, 3>{}); break;
-          default: ok = one_pass(std::integral_constant<int, 4>{}); break;
+          case 1: ok = want_score ? one_pass(std::integral_constant<int, 1>{}, sc_on)
+                                  : one_pass(std::integral_constant<int, 1>{}, sc_off); break;
+          case 2: ok = want_score ? one_pass(std::integral_constant<int, 2>{}, sc_on)
+                                  : one_pass(std::integral_constant<int, 2>{}, sc_off); break;
+          case 3: ok = want_score ? one_pass(std::integral_constant<int, 3>{}, sc_on)
+                                  : one_pass(std::integral_constant<int, 3>{}, sc_off); break;
+          default: ok = want_score ? one_pass(std::integral_constant<int, 4>{}, sc_on)
+                                   : one_pass(std::integral_constant<int, 4>{}, sc_off); break;
         }
         if (!ok) return false;
       } else {
@@ -455,8 +466,9 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
         // the probabilities, the sums and P (P chunk c lands on S columns
         // already read). The padding columns hold -inf from the mask step of
         // the S product and weight 0, so no key needs a test.
-        auto two_pass = [&](auto nc_tag) {
+        auto two_pass = [&](auto nc_tag, auto sc_tag) {
           constexpr int NC = decltype(nc_tag)::value;
+          constexpr bool SC = decltype(sc_tag)::value;
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c = 0; c < NC; ++c) {
@@ -486,9 +498,11 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
                         x0, x1);
               const float a = ex2_approx(x0), bb = ex2_approx(x1);
               const uint64_t e2 = f2_pack(a, bb);
-              const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
               lacc[i2 & 1] = f2_add(lacc[i2 & 1], e2);
-              sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+              if constexpr (SC) {
+                const float2 w2 = *reinterpret_cast<const float2*>(sw + j0);
+                sacc[i2 & 1] = f2_fma(f2_pack(w2.x, w2.y), e2, sacc[i2 & 1]);
+              }
               pk[i2] = pack_bf16x2(a, bb);
             }
             if (has_o) tmem_st16(tP + 16 * c, pk);
@@ -501,11 +515,17 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
           l = (l0 + l1) + (l2 + l3);
           score = (s0 + s1) + (s2 + s3);
         };
+        const std::true_type sc_on;
+        const std::false_type sc_off;
         switch (Lp / 32) {
-          case 5: two_pass(std::integral_constant<int, 5>{}); break;
-          case 6: two_pass(std::integral_constant<int, 6>{}); break;
-          case 7: two_pass(std::integral_constant<int, 7>{}); break;
-          default: two_pass(std::integral_constant<int, 8>{}); break;
+          case 5: want_score ? two_pass(std::integral_constant<int, 5>{}, sc_on)
+                             : two_pass(std::integral_constant<int, 5>{}, sc_off); break;
+          case 6: want_score ? two_pass(std::integral_constant<int, 6>{}, sc_on)
+                             : two_pass(std::integral_constant<int, 6>{}, sc_off); break;
+          case 7: want_score ? two_pass(std::integral_constant<int, 7>{}, sc_on)
+                             : two_pass(std::integral_constant<int, 7>{}, sc_off); break;
+          default: want_score ? two_pass(std::integral_constant<int, 8>{}, sc_on)
+                              : two_pass(std::integral_constant<int, 8>{}, sc_off); break;
         }
         if (!has_o) {
           tc_fence_before();
