@@ -773,33 +773,62 @@ def main():
     ev_in, ev_done, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_steps = max(4, args.steps)  # as many steps as the device-side measurement (fill and drain included)
+
+    def pipeline(n):
+        for i in range(n):
+            b = i % 2
+            ins, st = sets[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[b])  # step i-2 has finished reading this set
+                for n_, t in host.items():
+                    ins[n_].copy_(t, non_blocking=True)
+                ev_in[b].record(s_in)
+            comp.wait_event(ev_in[b])
+            if i >= 2:
+                comp.wait_event(ev_out[b])  # step i-2's results have left this set
+            st()
+            ev_done[b].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                for o, ho in zip(outs[b], host_out[b]):
+                    ho.copy_(o, non_blocking=True)
+                ev_out[b].record(s_out)
+
+    # untimed warm-up of the same pipeline (the first copies from freshly
+    # pinned pages run well below the link rate)
+    pipeline(args.warmup)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
     torch.cuda.synchronize()
     e0.record(s_in)
-    for i in range(e_steps):
-        b = i % 2
-        ins, st = sets[b]
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(ev_done[b])  # step i-2 has finished reading this set
-            for n, t in host.items():
-                ins[n].copy_(t, non_blocking=True)
-            ev_in[b].record(s_in)
-        comp.wait_event(ev_in[b])
-        if i >= 2:
-            comp.wait_event(ev_out[b])  # step i-2's results have left this set
-        st()
-        ev_done[b].record(comp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_done[b])
-            for o, ho in zip(outs[b], host_out[b]):
-                ho.copy_(o, non_blocking=True)
-            ev_out[b].record(s_out)
+    pipeline(e_steps)
     e1.record(s_out)
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / e_steps, dist, dev)
+    # the host link alone: one step's input and result copies, both
+    # directions at once, no compute (the bound the pipelined steps approach)
+    link = []
+    for _ in range(3):
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        c0.record(s_in)
+        with torch.cuda.stream(s_in):
+            for n_, t in host.items():
+                sets[0][0][n_].copy_(t, non_blocking=True)
+        s_out.wait_event(c0)
+        with torch.cuda.stream(s_out):
+            for o, ho in zip(outs[0], host_out[0]):
+                ho.copy_(o, non_blocking=True)
+        s_in.wait_stream(s_out)
+        c1.record(s_in)
+        torch.cuda.synchronize()
+        link.append(c0.elapsed_time(c1))
     e2e = {"value": job_throughput(world, f_step, ms_e2e), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": e_steps,
-           "overlap": "copies of step i overlap the compute of steps i-1 / i+1 (two buffer sets)"}
+           "overlap": "copies of step i overlap the compute of steps i-1 / i+1 (two buffer sets)",
+           "copies_alone_ms": min(link)}
     del sets, inp2, outs
 
     dense_list, srsu_list = step.launch_times()
