@@ -104,6 +104,7 @@ struct FlashParams {
   CUtensorMap qg_map[2];  // 2-D [B*N, H*D] gather map per chunk (rows of S)
   CUtensorMap k_map[2];   // 4-D [B, N, H, D]
   CUtensorMap v_map;      // 4-D [B, N, H, D] V map, box kVW wide (chunk chosen by x)
+  CUtensorMap o_map[2];   // 4-D [B, n_q, H, D] map of O per chunk (output tile stores)
   const int32_t* S;       // [B, n_q] query rows when gathering, else null
   __nv_bfloat16* O;       // [B, n_q, H, D]
   float* lse;             // [B, H, n_q] or null
@@ -727,26 +728,44 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
     const bool have_o = ok && warp_wait(&o_full[t], 0, &abort_flag);
     if (have_o) tc_fence_after();
     const bool valid = q_row < p.n_q;
-    __nv_bfloat16* orow = p.O + ((static_cast<size_t>(b) * p.n_q + (valid ? q_row : 0)) * p.H + h) * D + DH * hf;
-    if (have_o && !partial) {
-      const float inv_l = 1.f / l;
+    if (!partial) {
+      // O / l in bf16 into this tile's query buffer (free: every S product
+      // of the tile completed before its last P V), laid out as the query
+      // tile was, then one TMA store per head-dim chunk; rows past n_q are
+      // clipped by the store
+      uint8_t* stage = sQ + t * TB;
+      if (have_o) {
+        const float inv_l = 1.f / l;
 #pragma unroll
-      for (int c = 0; c < DH / 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(tO + 16 * c, o);
-        tmem_ld_wait16(o);
-        uint32_t pk[8];
+        for (int c = 0; c < DH / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16 * c, o);
+          tmem_ld_wait16(o);
+          uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int i = 0; i < 8; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int u = (DH * hf + 16 * c) / 8 + v;  // 16-byte unit of the row
+            const int cq = u >> 3, uc = u & 7;
+            const int rb = C::row_bytes(cq);
+            const int xr = rb == 128 ? (row & 7) : ((row >> 1) & 3);
+            *reinterpret_cast<uint4*>(stage + C::chunk_off(cq) + row * rb + ((uc ^ xr) << 4)) =
+                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
+        if (valid && hf == 0 && p.lse != nullptr)
+          p.lse[(static_cast<size_t>(b) * p.H + h) * p.n_q + q_row] = (m_use + __log2f(l)) * 0.69314718055994531f;
       }
-      if (valid && hf == 0 && p.lse != nullptr)
-        p.lse[(static_cast<size_t>(b) * p.H + h) * p.n_q + q_row] = (m_use + __log2f(l)) * 0.69314718055994531f;
+      fence_proxy_async_smem();
+      named_bar_sync(10 + t, 256);  // the tile's eight softmax warps
+      if (quarter == 0 && hf == 0 && lane == 0 && !abort_flag && q_base + t * 128 < p.n_q) {
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_store_4d(&p.o_map[c], stage + C::chunk_off(c), 64 * c, h, q_base + t * 128, b);
+        bulk_commit_group();
+        bulk_wait_read_all();
+      }
     }
     if (partial) {
       // one part of a split unit: store the unnormalised O row with its

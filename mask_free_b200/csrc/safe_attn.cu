@@ -347,6 +347,7 @@ bool fill_srsu(FlashParams& p, const void* Q, int q_compact, const int32_t* S, i
     bool ok = encode_rows_map(&p.k_map[c], Kc, B, N, H, d, c);
     ok = ok && (q_compact ? encode_rows_map(&p.q_map[c], Q, B, k, H, d, c)
                           : encode_gather_map(&p.qg_map[c], Q, B, N, H, d, c));
+    ok = ok && encode_rows_map(&p.o_map[c], O_S, B, k, H, d, c);
     if (!ok) return false;
   }
   p.S = S;
@@ -463,7 +464,8 @@ safe_status safe_attn_self(const void* Q, const void* K, const void* V, void* O,
   if (!supported_d(d)) return SAFE_ERR_UNSUPPORTED;
   FlashParams p{};
   for (int c = 0; c < nchunks(d); ++c) {
-    if (!encode_rows_map(&p.q_map[c], Q, B, N, H, d, c) || !encode_rows_map(&p.k_map[c], K, B, N, H, d, c))
+    if (!encode_rows_map(&p.q_map[c], Q, B, N, H, d, c) || !encode_rows_map(&p.k_map[c], K, B, N, H, d, c) ||
+        !encode_rows_map(&p.o_map[c], O, B, N, H, d, c))
       return SAFE_ERR_CUDA;
   }
   if (!encode_v_map(&p.v_map, V, B, N, H, d)) return SAFE_ERR_CUDA;
