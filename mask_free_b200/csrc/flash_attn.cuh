@@ -142,6 +142,9 @@ __host__ __device__ constexpr int flash_smem_bytes() {
   return 1024 /*align slack*/ + (2 + 2 * C::kStages) * C::kTileBytes + 512 /*barriers + tmem slot*/;
 }
 
+// Most key-range parts a split unit is cut into (the planner's limit).
+constexpr int kMaxSplit = 16;
+
 // Combines the key-range parts of the split units: one warp per query row,
 // lane l owns columns [4l, 4l + 4):
 //   M = max_i m_i,  L = sum_i 2^(m_i - M) l_i,  O = sum_i 2^(m_i - M) O_i / L
@@ -156,23 +159,35 @@ __global__ void __launch_bounds__(256) flash_merge_kernel(const __grid_constant_
   const int qr = (unit % p.n_mblk) * 256 + r;
   if (qr >= p.n_q) return;
   const size_t slot0 = static_cast<size_t>(tu) * p.split * 256 + r;
+  // every part's (m, l) and O slice requested at once (at most kMaxSplit
+  // parts), then combined
+  const bool active = lane < D / 4;
+  float2 ml[kMaxSplit];
+  float4 x[kMaxSplit];
+#pragma unroll
+  for (int i = 0; i < kMaxSplit; ++i) {
+    ml[i] = make_float2(-INFINITY, 0.f);
+    x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < p.split) {
+      const size_t slot = slot0 + static_cast<size_t>(i) * 256;
+      ml[i] = __ldcg(&p.ws_ml[slot]);
+      if (active) x[i] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + slot * D) + lane);
+    }
+  }
   float M = -INFINITY;
-  for (int i = 0; i < p.split; ++i) M = fmaxf(M, __ldcg(&p.ws_ml[slot0 + static_cast<size_t>(i) * 256]).x);
+#pragma unroll
+  for (int i = 0; i < kMaxSplit; ++i) M = fmaxf(M, ml[i].x);
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const bool active = lane < D / 4;
-#pragma unroll 4
-  for (int i = 0; i < p.split; ++i) {
-    const size_t slot = slot0 + static_cast<size_t>(i) * 256;
-    const float2 ml = __ldcg(&p.ws_ml[slot]);
-    const float w = ex2_approx(ml.x - M);
-    L = fmaf(w, ml.y, L);
-    if (active) {
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(p.ws_o + slot * D) + lane);
-      acc.x = fmaf(w, x.x, acc.x);
-      acc.y = fmaf(w, x.y, acc.y);
-      acc.z = fmaf(w, x.z, acc.z);
-      acc.w = fmaf(w, x.w, acc.w);
+#pragma unroll
+  for (int i = 0; i < kMaxSplit; ++i) {
+    if (i < p.split) {
+      const float w = ex2_approx(ml[i].x - M);
+      L = fmaf(w, ml[i].y, L);
+      acc.x = fmaf(w, x[i].x, acc.x);
+      acc.y = fmaf(w, x[i].y, acc.y);
+      acc.z = fmaf(w, x[i].z, acc.z);
+      acc.w = fmaf(w, x[i].w, acc.w);
     }
   }
   const float inv_l = 1.f / L;

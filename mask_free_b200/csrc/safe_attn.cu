@@ -162,7 +162,7 @@ FlashPlan plan_flash(int B, int H, int n_q, int N, int d, int sms) {
   // tiles.
   const double whole = n_kv + 2.0;
   double best = static_cast<double>((pl.units + sms - 1) / sms) * whole;
-  const int max_split = n_kv / 4 < 16 ? n_kv / 4 : 16;
+  const int max_split = n_kv / 4 < kMaxSplit ? n_kv / 4 : kMaxSplit;  // the merge kernel takes at most kMaxSplit parts
   for (int fw = pl.units / sms; fw >= 0 && fw >= pl.units / sms - 1; --fw) {
     const int f = fw * sms, r = pl.units - f;
     if (r <= 0) continue;
