@@ -88,7 +88,9 @@ __host__ __device__ constexpr int cross_smem_bytes(int M) {
                                                                   : cross_smem_need<D>(M, cross_slots<D>(M));
 }
 
-template <int D, bool kSep>
+// kO: O is written (cross-attention); otherwise only the PCSP partials
+// (p.O == nullptr), and the softmax builds no P.
+template <int D, bool kSep, bool kO>
 __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __grid_constant__ CrossParams p) {
   using C = TileCfg<D>;
   constexpr int TB = C::kTileBytes;
@@ -128,7 +130,9 @@ __global__ void __launch_bounds__(kCrossThreads, 1) cross_attn_kernel(const __gr
   const int tile1 = tile0 + per < n_tiles ? tile0 + per : n_tiles;
   if (tile0 >= tile1) return;  // uniform for the CTA, before any barrier or TMEM use
   const int n_my = tile1 - tile0;
-  const bool has_o = p.O != nullptr;
+  // (runtime for kO: the O-writing kernel compiles as it did with one
+  // instantiation for both uses, which its register allocation prefers)
+  const bool has_o = kO && p.O != nullptr;
 
   int L = __ldg(p.valid_len + b);
   if (L < 1 || L > p.M) {

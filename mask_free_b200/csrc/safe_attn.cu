@@ -228,17 +228,23 @@ safe_status dispatch_flash(int d, FlashParams& p, void* ws, size_t ws_bytes, cud
   }
 }
 
+template <int D, bool kSep, bool kO>
+cudaError_t cross_smem_attr() {
+  return cudaFuncSetAttribute(cross_attn_kernel<D, kSep, kO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kCrossMaxSmem);
+}
+
 template <int D>
 safe_status launch_cross(CrossParams& p, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(cross_attn_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kCrossMaxSmem);
-    if constexpr (D <= 96)
-      if (attr_err == cudaSuccess)
-        attr_err = cudaFuncSetAttribute(cross_attn_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kCrossMaxSmem);
+    attr_err = cross_smem_attr<D, false, true>();
+    if (attr_err == cudaSuccess) attr_err = cross_smem_attr<D, false, false>();
+    if constexpr (D <= 96) {
+      if (attr_err == cudaSuccess) attr_err = cross_smem_attr<D, true, true>();
+      if (attr_err == cudaSuccess) attr_err = cross_smem_attr<D, true, false>();
+    }
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   // one CTA per SM (each holds all of TMEM), a few per (b, h), each streaming
@@ -248,14 +254,24 @@ safe_status launch_cross(CrossParams& p, cudaStream_t s) {
   per_bh = per_bh < 1 ? 1 : (per_bh > n_tiles ? n_tiles : per_bh);
   p.qs = cross_slots<D>(p.M);
   dim3 grid(per_bh, p.H, p.B);
-  bool launched = false;
+  const int smem = cross_smem_bytes<D>(p.M);
+  const bool o = p.O != nullptr;  // else PCSP partials only
+  bool sep = false;
+  if constexpr (D <= 96) sep = cross_sep_p<D>(p.M);
   if constexpr (D <= 96) {
-    if (cross_sep_p<D>(p.M)) {
-      cross_attn_kernel<D, true><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
-      launched = true;
+    if (sep) {
+      if (o)
+        cross_attn_kernel<D, true, true><<<grid, kCrossThreads, smem, s>>>(p);
+      else
+        cross_attn_kernel<D, true, false><<<grid, kCrossThreads, smem, s>>>(p);
     }
   }
-  if (!launched) cross_attn_kernel<D, false><<<grid, kCrossThreads, cross_smem_bytes<D>(p.M), s>>>(p);
+  if (!sep) {
+    if (o)
+      cross_attn_kernel<D, false, true><<<grid, kCrossThreads, smem, s>>>(p);
+    else
+      cross_attn_kernel<D, false, false><<<grid, kCrossThreads, smem, s>>>(p);
+  }
   return launch_status();
 }
 
