@@ -196,6 +196,7 @@ safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   FlashPlan pl = plan_flash(p.B, p.H, p.n_q, p.N, D, device_sms());
+  if (pl.split > kMaxSplit) return SAFE_ERR_UNSUPPORTED;  // the merge takes at most kMaxSplit parts
   if (pl.split > 1 && (ws == nullptr || ws_bytes < pl.ws_bytes)) {
     pl.full = pl.units;  // no workspace: whole units only
     pl.split = 1;
