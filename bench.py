@@ -888,9 +888,9 @@ def main():
 
     dense_list, srsu_list = step.launch_times()
     dense_ms, srsu_ms = statistics.mean(dense_list), statistics.mean(srsu_list)
-    # the step is milliseconds long and the timed region well under a second:
-    # the burst bf16 peak is the denominator (the sustained figure applies to
-    # a kernel timed inside a seconds-long loop)
+    # the burst bf16 peak is the denominator (the larger, so the smaller
+    # fraction); the fraction of the sustained peak, measured over a
+    # seconds-long GEMM loop under the power cap, is printed beside it
     achieved = f_dense / (dense_ms * 1e-3) / 1e12
     achieved_srsu = f_srsu / (srsu_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
