@@ -150,6 +150,7 @@ constexpr int kMaxSplit = 16;
 //   M = max_i m_i,  L = sum_i 2^(m_i - M) l_i,  O = sum_i 2^(m_i - M) O_i / L
 template <int D>
 __global__ void __launch_bounds__(256) flash_merge_kernel(const __grid_constant__ FlashParams p, int tail_units) {
+  pdl_wait();  // every part of the attention launch is stored
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (wid >= tail_units * 256) return;
@@ -404,6 +405,10 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // launched as a programmatic dependent: the set-up above overlapped the
+  // previous kernel; its outputs (the inputs here) are read only from now on
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp < 4) {
     regs_dealloc<kFlashRegsControl>();

@@ -60,6 +60,7 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ S,
                                                           uint4* __restrict__ Xg, int B, int N, int k,
                                                           int units_per_row) {
+  pdl_launch_dependents();  // a dependent attention kernel may set up meanwhile
   const int lane = threadIdx.x & 31;
   const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (w >= static_cast<long long>(B) * k) return;

@@ -213,8 +213,26 @@ safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t
     p.ws_ml = reinterpret_cast<float2*>(w + pl.ws_ml);
   }
   const unsigned grid = static_cast<unsigned>(pl.full + pl.tail * pl.split);
-  flash_fwd_kernel<D, kAsm><<<grid, kFlashThreads, smem, s>>>(p);
-  if (pl.split > 1) flash_merge_kernel<D><<<(pl.tail * 256 + 7) / 8, 256, 0, s>>>(p, pl.tail);
+  // both launches are programmatic dependents of what precedes them in the
+  // stream: their set-up overlaps its tail, and each waits (griddepcontrol)
+  // for it before reading anything
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kFlashThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, flash_fwd_kernel<D, kAsm>, p) != cudaSuccess) return SAFE_ERR_CUDA;
+  if (pl.split > 1) {
+    cfg.gridDim = dim3((pl.tail * 256 + 7) / 8);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, flash_merge_kernel<D>, p, pl.tail) != cudaSuccess) return SAFE_ERR_CUDA;
+  }
   return launch_status();
 }
 
