@@ -420,16 +420,19 @@ def kernel_table(dev, pk):
             if side * side == s.N:
                 sf = torch.empty_like(sc)
                 wsf = torch.empty(ops.sensitivity_workspace_bytes(s.B, s.N), dtype=torch.uint8, device=dev)
-                t_f = time_flushed(lambda: ops.sensitivity_field(sc, side, side, 2.0, out=sf, ws=wsf))
+                f_f = lambda: ops.sensitivity_field(sc, side, side, 2.0, out=sf, ws=wsf)
+                t_f = time_flushed(f_f)
                 out["sensitivity_field"] = {"ms": t_f, "grid": f"{side}x{side}", "sigma": 2.0,
-                                            "gbs": 5 * 4 * s.B * s.N / t_f / 1e6}
+                                            "gbs": 5 * 4 * s.B * s.N / t_f / 1e6, "ms_back_to_back": time_kernel(f_f)}
                 for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
                     fc = torch.randn((1, s.N, 16), device=dev).to(dt)
                     fu = torch.randn((1, s.N, 16), device=dev).to(dt)
                     fo = torch.empty_like(fc)
-                    t_g = time_flushed(lambda: ops.sw_cfg(fc, fu, sf[:1], 4.0, 7.5, out=fo))
+                    f_g = lambda: ops.sw_cfg(fc, fu, sf[:1], 4.0, 7.5, out=fo)
+                    t_g = time_flushed(f_g)
                     gb = 3 * fc.numel() * fc.element_size() + 4 * s.N
-                    out[f"sw_cfg_{tag}"] = {"ms": t_g, "gbs": gb / t_g / 1e6, "pct_hbm": 100 * gb / t_g / 1e6 / pk["hbm"]}
+                    out[f"sw_cfg_{tag}"] = {"ms": t_g, "gbs": gb / t_g / 1e6, "pct_hbm": 100 * gb / t_g / 1e6 / pk["hbm"],
+                                            "ms_back_to_back": time_kernel(f_g)}
             # SRSU wall time against |S|/N
             sweep = {}
             for rho in (0.1, 0.2, 0.3, 0.5, 1.0):
