@@ -333,6 +333,9 @@ safe_status safe_sw_cfg(const void* f_c, const void* f_u, const float* s, void* 
  *        a compact [B, k, d_in] matrix, which the GEMM then reads by tiled
  *        copies. NULL (or ws_bytes too small): the GEMM gathers the rows of
  *        S itself, correct but slower. Ignored when S == NULL.
+ *        Every row (S == NULL or the compact copy) runs on CTA pairs
+ *        (clusters of two SMs, 256 x 256 output tiles); the gathered form
+ *        on single SMs (128 x 256 tiles). Both give the same bits.
  *  d_in >= 64 and d_out >= 8, both multiples of 8; X, Wt, Y 16-byte aligned.
  */
 size_t safe_gather_linear_workspace_bytes(int B, int k, int d_in);

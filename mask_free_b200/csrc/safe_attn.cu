@@ -751,13 +751,17 @@ safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const voi
     S = nullptr;
   }
   const int R = S != nullptr ? k : N;
-  const int64_t m_tiles = (R + 127) / 128, n_tiles = (d_out + 255) / 256;
+  // plain rows: CTA pairs on 256 x 256 tiles; rows of S gathered in the
+  // kernel (no workspace): one CTA per 128 x 256 tile
+  const bool pairs = S == nullptr;
+  const int64_t m_tiles = (R + (pairs ? 255 : 127)) / (pairs ? 256 : 128), n_tiles = (d_out + 255) / 256;
   const int64_t tiles = static_cast<int64_t>(B) * m_tiles * n_tiles;
   if (tiles > INT_MAX) return SAFE_ERR_UNSUPPORTED;
   LinearParams p{};
   if (!encode_matrix_map(&p.x_map, X, static_cast<uint64_t>(d_in), static_cast<uint64_t>(B) * N, 64, 1) ||
       !encode_matrix_map(&p.xt_map, X, static_cast<uint64_t>(d_in), static_cast<uint64_t>(B) * N, 64, 128) ||
-      !encode_matrix_map(&p.w_map, Wt, static_cast<uint64_t>(d_in), static_cast<uint64_t>(d_out), 64, 256))
+      !encode_matrix_map(&p.w_map, Wt, static_cast<uint64_t>(d_in), static_cast<uint64_t>(d_out), 64, 256) ||
+      !encode_matrix_map(&p.w2_map, Wt, static_cast<uint64_t>(d_in), static_cast<uint64_t>(d_out), 64, 128))
     return SAFE_ERR_CUDA;
   p.S = S;
   p.bias = bias;
@@ -775,11 +779,18 @@ safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const voi
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(linear_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLin2Smem);
   });
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   const int sms = device_sms();
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  linear_kernel<<<grid, kLinThreads, kLinSmem, as_stream(stream)>>>(p);
+  if (pairs) {
+    const int n_pairs = static_cast<int>(tiles < sms / 2 ? tiles : sms / 2);
+    linear_pair_kernel<<<2 * (n_pairs > 0 ? n_pairs : 1), kLinThreads, kLin2Smem, as_stream(stream)>>>(p);
+  } else {
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    linear_kernel<<<grid, kLinThreads, kLinSmem, as_stream(stream)>>>(p);
+  }
   return launch_status();
 }
 

@@ -74,6 +74,24 @@ def test_gather_linear_parity(B, N, d_in, d_out, k, act, with_bias, compact_copy
     assert ops.device_status() == 0
 
 
+def test_gelu_over_the_whole_pre_activation_range():
+    # pre-activations from -12 to 12 through the bias: GELU's tails (y -> -0
+    # for very negative inputs, y -> x for large ones) against the oracle's
+    # tanh form, on both kernels (every row: CTA pairs; rows of S gathered
+    # by the GEMM: one CTA per tile)
+    B, N, d_in, d_out = 1, 300, 64, 512
+    X, Wt, _ = _layer(B, N, d_in, d_out, seed=31)
+    bias = torch.linspace(-12.0, 12.0, d_out)
+    Xd, Wd, bd = X.to(DEV), Wt.to(DEV), bias.to(DEV)
+    S = _rows(B, N, 150, seed=4)
+    X64 = to64(X)
+    got = ops.gather_linear(Xd, Wd, bias=bd, act="gelu_tanh")
+    _check(got, X64, to64(Wt), bias.numpy().astype(np.float64), "gelu_tanh")
+    got = ops.gather_linear(Xd, Wd, S=torch.from_numpy(S).to(DEV), bias=bd, act="gelu_tanh", ws=False)
+    _check(got, np.stack([X64[0, S[0]]]), to64(Wt), bias.numpy().astype(np.float64), "gelu_tanh")
+    assert ops.device_status() == 0
+
+
 def test_gathered_rows_equal_dense_rows_bitwise():
     B, N, d_in, d_out, k = 2, 700, 320, 520, 211
     X, Wt, bias = _layer(B, N, d_in, d_out, seed=17)
