@@ -785,7 +785,21 @@ safe_status safe_gather_linear(const void* X, const int32_t* S, int k, const voi
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   const int sms = device_sms();
   if (pairs) {
-    const int n_pairs = static_cast<int>(tiles < sms / 2 ? tiles : sms / 2);
+    // as many pairs as can be resident at once (a GPC with an odd number of
+    // free SMs leaves one of them out), so that every pair starts at once
+    static int max_pairs[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int& mp = max_pairs[dev >= 0 && dev < 64 ? dev : 0];
+    if (mp == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(2 * (sms / 2)));
+      cfg.blockDim = dim3(kLinThreads);
+      cfg.dynamicSmemBytes = kLin2Smem;
+      int n = 0;
+      mp = cudaOccupancyMaxActiveClusters(&n, linear_pair_kernel, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
+    }
+    const int n_pairs = static_cast<int>(tiles < mp ? tiles : mp);
     linear_pair_kernel<<<2 * (n_pairs > 0 ? n_pairs : 1), kLinThreads, kLin2Smem, as_stream(stream)>>>(p);
   } else {
     const int grid = static_cast<int>(tiles < sms ? tiles : sms);

@@ -402,71 +402,4 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// ---------------------------------------------------------------- CTA pairs (cta_group::2)
-// Rank of this CTA in its cluster.
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// shared::cluster address of shared-memory location `p` in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-// Every thread of both CTAs of the cluster arrives and waits.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Arrive on an mbarrier given by its shared::cluster address (any CTA of the cluster).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-}
-// TMEM of a CTA pair: one warp of each CTA of the pair (the same warp index
-// in both) allocates and frees, with the same destination slot.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// Pair MMA, issued by the even CTA: D (M = 256: rows 0..127 in the even CTA's
-// TMEM, 128..255 in the odd one's) (+)= A B^T, A's rows and B's rows (the
-// N columns) split in halves between the two CTAs' shared memory at the
-// same offsets as the descriptors give.
-__device__ __forceinline__ void umma_pair_ss_if(uint32_t leader, uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 e, %5, 0;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(leader)
-      : "memory");
-}
-// Arrive on the mbarrier at shared::cluster address `caddr` (either CTA of
-// the pair) once the pair MMAs this thread issued so far have completed.
-__device__ __forceinline__ void umma_pair_commit_if(uint32_t leader, uint32_t caddr) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "setp.ne.b32 e, %1, 0;\n\t"
-      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(caddr),
-      "r"(leader)
-      : "memory");
-}
-// 2-D tiled TMA load into this CTA's shared memory whose completion is
-// counted on the mbarrier at shared::cluster address `mbar` (the pair's
-// even CTA), box set by the tensor map.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t mbar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar), "r"(c0), "r"(c1)
-      : "memory");
-}
-
 }  // namespace safe
