@@ -17,8 +17,9 @@
 //              issues): tcgen05.mma M = 128, N = 256, K = 16 into one of
 //              two 256-column TMEM accumulators (tile i uses buffer i & 1)
 //   warp 2     TMEM allocation
-//   warps 4..7 epilogue: tcgen05.ld of the accumulator (TMEM lane = row of
-//              the tile), + bias, activation, bf16 rows to global memory;
+//   warps 4..11 epilogue: tcgen05.ld of the accumulator (TMEM lane = row of
+//              the tile; warps 4..7 columns 0..127, warps 8..11 columns
+//              128..255), + bias, activation, bf16 rows to global memory;
 //              the buffer is released once read, so the next tile's MMAs
 //              overlap this tile's stores
 // Every wait is bounded (sm100.cuh); a row index outside [0, N) is flagged
@@ -110,7 +111,7 @@ struct LinearParams {
   int tiles;            // B * m_tiles * n_tiles
 };
 
-constexpr int kLinThreads = 256;
+constexpr int kLinThreads = 384;  // warps 0-3 producer / MMA / TMEM, warps 4-11 epilogue
 constexpr int kLinStages = 4;
 constexpr int kLinABytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kLinBBytes = 256 * 128;  // 256 rows x 64 bf16
@@ -147,6 +148,67 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
   for (int u = lane; u < units_per_row; u += 32) dst[u] = __ldg(src + u);
 }
 
+// Epilogue of one output tile, run by eight warps: warp 4 + 4e + q reads
+// TMEM lanes 32q .. 32q + 31 (rows of the tile) and columns
+// [128e, 128e + 128) of the accumulator at `tacc` (four 32-column chunks),
+// adds the bias, applies the activation and stores bf16 into `yrow` (the
+// tile row's output, columns from n0). `release` is called once this
+// thread's last chunk is in registers (the accumulator may then be reused).
+template <typename Release>
+__device__ __forceinline__ void linear_epilogue_tile(const LinearParams& p, uint32_t tacc, int e, int n0,
+                                                     __nv_bfloat16* yrow, bool valid, Release release) {
+  const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0;
+#pragma unroll 1
+  for (int c = 4 * e; c < 4 * e + 4; ++c) {
+    uint32_t v[32];
+    tmem_ld32(tacc + 32 * c, v);
+    tmem_ld_wait32(v);
+    if (c == 4 * e + 3) {
+      tc_fence_before();
+      release();
+    }
+    const int nc = n0 + 32 * c;
+    if (nc >= p.d_out) continue;
+    // the chunk's 32 bias values: 8 vector loads (the same for every row,
+    // so they come from L1), or element by element at the ragged last chunk
+    // or a bias that is not 16-byte aligned
+    float bv[32];
+    if (p.bias == nullptr) {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) bv[k] = 0.f;
+    } else if (bias_vec && nc + 32 <= p.d_out) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + nc) + u);
+        bv[4 * u] = b4.x;
+        bv[4 * u + 1] = b4.y;
+        bv[4 * u + 2] = b4.z;
+        bv[4 * u + 3] = b4.w;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) bv[k] = nc + k < p.d_out ? __ldg(p.bias + nc + k) : 0.f;
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float f0 = __uint_as_float(v[2 * k]) + bv[2 * k], f1 = __uint_as_float(v[2 * k + 1]) + bv[2 * k + 1];
+      if (p.act == 1) {
+        f0 = gelu_tanh_f(f0);
+        f1 = gelu_tanh_f(f1);
+      }
+      pk[k] = pack_bf16x2(f0, f1);
+    }
+    if (valid) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (nc + 8 * u < p.d_out)
+          *reinterpret_cast<uint4*>(yrow + nc + 8 * u) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
+                                                                    pk[4 * u + 3]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_constant__ LinearParams p) {
   constexpr int ST = kLinStages;
   extern __shared__ uint8_t smem_raw[];
@@ -176,7 +238,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);  // every epilogue thread
+      mbar_init(&acc_empty[a], 256);  // every epilogue thread
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -281,9 +343,8 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3, row = q * 32 + lane;
+    const int q = warp & 3, row = q * 32 + lane, e = (warp - 4) >> 2;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0;
     for (int i = 0; i < n_local; ++i) {
       const int a = i & 1;
       if (!warp_wait(&acc_full[a], (i >> 1) & 1, &abort_flag)) break;
@@ -293,57 +354,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
       const int r = r0 + row;
       const bool valid = r < p.R;
       __nv_bfloat16* yrow = p.Y + (static_cast<size_t>(b) * p.R + (valid ? r : 0)) * p.d_out;
-      const uint32_t tacc = tbase + lane_addr + 256u * a;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tacc + 32 * c, v);
-        tmem_ld_wait32(v);
-        if (c == 7) {
-          // the whole accumulator is in registers or stored: release it
-          tc_fence_before();
-          mbar_arrive(&acc_empty[a]);
-        }
-        const int nc = n0 + 32 * c;
-        if (nc >= p.d_out) continue;
-        // the chunk's 32 bias values: 8 vector loads (the same for every
-        // row, so they come from L1), or element by element at the ragged
-        // last chunk or a bias that is not 16-byte aligned
-        float bv[32];
-        if (p.bias == nullptr) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) bv[e] = 0.f;
-        } else if (bias_vec && nc + 32 <= p.d_out) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + nc) + u);
-            bv[4 * u] = b4.x;
-            bv[4 * u + 1] = b4.y;
-            bv[4 * u + 2] = b4.z;
-            bv[4 * u + 3] = b4.w;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) bv[e] = nc + e < p.d_out ? __ldg(p.bias + nc + e) : 0.f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float f0 = __uint_as_float(v[2 * e]) + bv[2 * e], f1 = __uint_as_float(v[2 * e + 1]) + bv[2 * e + 1];
-          if (p.act == 1) {
-            f0 = gelu_tanh_f(f0);
-            f1 = gelu_tanh_f(f1);
-          }
-          pk[e] = pack_bf16x2(f0, f1);
-        }
-        if (valid) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (nc + 8 * u < p.d_out)
-              *reinterpret_cast<uint4*>(yrow + nc + 8 * u) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                                                                        pk[4 * u + 3]);
-        }
-      }
+      linear_epilogue_tile(p, tbase + lane_addr + 256u * a, e, n0, yrow, valid, [&] { mbar_arrive(&acc_empty[a]); });
     }
   }
 
@@ -366,11 +377,11 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_kernel(const __grid_con
 //              chunk, counted on the even CTA's stage barrier
 //   warp 1     MMA issuer (even CTA only)
 //   warp 2     TMEM allocation (both CTAs, pair form)
-//   warps 4..7 epilogue in both CTAs (the CTA's 128 rows)
+//   warps 4..11 epilogue in both CTAs (the CTA's 128 rows, two column halves)
 // Barriers: full[s] of the even CTA takes both CTAs' copies (64 KB);
 // empty[s] of each CTA is arrived on by the even CTA's MMA commit (the
 // stage of both CTAs may be refilled); acc_full[a] the same for the
-// accumulator; acc_empty[a] of the even CTA counts the 256 epilogue threads
+// accumulator; acc_empty[a] of the even CTA counts the 512 epilogue threads
 // of the pair once they have read the accumulator. Every wait is bounded.
 constexpr int kLin2Stages = 6;
 constexpr int kLin2ABytes = 128 * 128;  // 128 rows x 64 bf16
@@ -407,7 +418,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kLinThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 256);  // every epilogue thread of both CTAs
+      mbar_init(&acc_empty[a], 512);  // every epilogue thread of both CTAs
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -508,9 +519,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kLinThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3, row = q * 32 + lane;
+    const int q = warp & 3, row = q * 32 + lane, e = (warp - 4) >> 2;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0;
     const uint32_t acce0 = cluster_addr(acc_empty, 0);
     for (int i = 0; i < n_local; ++i) {
       const int a = i & 1;
@@ -521,55 +531,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kLinThreads, 1)
       const int r = r0 + 128 * static_cast<int>(rank) + row;
       const bool valid = r < p.R;
       __nv_bfloat16* yrow = p.Y + (static_cast<size_t>(b) * p.R + (valid ? r : 0)) * p.d_out;
-      const uint32_t tacc = tbase + lane_addr + 256u * a;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tacc + 32 * c, v);
-        tmem_ld_wait32(v);
-        if (c == 7) {
-          // the whole accumulator is in registers or stored: release it to
-          // the even CTA's issuer
-          tc_fence_before();
-          mbar_arrive_cluster(acce0 + static_cast<uint32_t>(a * sizeof(uint64_t)));
-        }
-        const int nc = n0 + 32 * c;
-        if (nc >= p.d_out) continue;
-        float bv[32];
-        if (p.bias == nullptr) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) bv[e] = 0.f;
-        } else if (bias_vec && nc + 32 <= p.d_out) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + nc) + u);
-            bv[4 * u] = b4.x;
-            bv[4 * u + 1] = b4.y;
-            bv[4 * u + 2] = b4.z;
-            bv[4 * u + 3] = b4.w;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) bv[e] = nc + e < p.d_out ? __ldg(p.bias + nc + e) : 0.f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float f0 = __uint_as_float(v[2 * e]) + bv[2 * e], f1 = __uint_as_float(v[2 * e + 1]) + bv[2 * e + 1];
-          if (p.act == 1) {
-            f0 = gelu_tanh_f(f0);
-            f1 = gelu_tanh_f(f1);
-          }
-          pk[e] = pack_bf16x2(f0, f1);
-        }
-        if (valid) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (nc + 8 * u < p.d_out)
-              *reinterpret_cast<uint4*>(yrow + nc + 8 * u) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                                                                        pk[4 * u + 3]);
-        }
-      }
+      // the accumulator is released to the even CTA's issuer
+      linear_epilogue_tile(p, tbase + lane_addr + 256u * a, e, n0, yrow, valid,
+                           [&] { mbar_arrive_cluster(acce0 + static_cast<uint32_t>(a * sizeof(uint64_t))); });
     }
   }
 
