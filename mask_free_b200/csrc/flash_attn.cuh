@@ -122,8 +122,12 @@ struct FlashParams {
   // CTA each, whose partial results flash_merge_kernel combines (balances
   // the last, partial wave of CTAs).
   int n_mblk, full_units, split;
-  float* ws_o;            // [tail units][split][256][D] unnormalised partial O
-  float2* ws_ml;          // [tail units][split][256] (running max in log2 units, row sum)
+  // part `part` of tail unit `tu` is slot tu * split + part: its rows' O / l
+  // in bf16 ([slots * 256, D], written by TMA stores through ws_map, a 4-D
+  // [1, slots * 256, 1, D] view) and (running max in log2 units, row sum)
+  __nv_bfloat16* ws_ob;
+  float2* ws_ml;
+  CUtensorMap ws_map[2];
 };
 
 constexpr int kFlashThreads = 640;
@@ -164,31 +168,32 @@ __global__ void __launch_bounds__(256) flash_merge_kernel(const __grid_constant_
   // parts), then combined
   const bool active = lane < D / 4;
   float2 ml[kMaxSplit];
-  float4 x[kMaxSplit];
+  uint2 x[kMaxSplit];  // four bf16 of O_i / l_i
 #pragma unroll
   for (int i = 0; i < kMaxSplit; ++i) {
     ml[i] = make_float2(-INFINITY, 0.f);
-    x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    x[i] = make_uint2(0u, 0u);
     if (i < p.split) {
       const size_t slot = slot0 + static_cast<size_t>(i) * 256;
       ml[i] = __ldcg(&p.ws_ml[slot]);
-      if (active) x[i] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + slot * D) + lane);
+      if (active) x[i] = __ldcg(reinterpret_cast<const uint2*>(p.ws_ob + slot * D) + lane);
     }
   }
   float M = -INFINITY;
 #pragma unroll
   for (int i = 0; i < kMaxSplit; ++i) M = fmaxf(M, ml[i].x);
+  // O = sum_i 2^(m_i - M) l_i (O_i / l_i) / L,  L = sum_i 2^(m_i - M) l_i
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < kMaxSplit; ++i) {
     if (i < p.split) {
-      const float w = ex2_approx(ml[i].x - M);
-      L = fmaf(w, ml[i].y, L);
-      acc.x = fmaf(w, x[i].x, acc.x);
-      acc.y = fmaf(w, x[i].y, acc.y);
-      acc.z = fmaf(w, x[i].z, acc.z);
-      acc.w = fmaf(w, x[i].w, acc.w);
+      const float w = ex2_approx(ml[i].x - M) * ml[i].y;
+      L += w;
+      acc.x = fmaf(w, __uint_as_float(x[i].x << 16), acc.x);
+      acc.y = fmaf(w, __uint_as_float(x[i].x & 0xFFFF0000u), acc.y);
+      acc.z = fmaf(w, __uint_as_float(x[i].y << 16), acc.z);
+      acc.w = fmaf(w, __uint_as_float(x[i].y & 0xFFFF0000u), acc.w);
     }
   }
   const float inv_l = 1.f / L;
@@ -748,12 +753,15 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
     const bool have_o = ok && warp_wait(&o_full[t], 0, &abort_flag);
     if (have_o) tc_fence_after();
     const bool valid = q_row < p.n_q;
-    if (!partial) {
+    {
       // O / l in bf16 into this tile's query buffer (free: every S product
       // of the tile completed before its last P V), laid out as the query
-      // tile was, then one TMA store per head-dim chunk; rows past n_q are
-      // clipped by the store
+      // tile was, then one TMA store per head-dim chunk: into O (rows past
+      // n_q are clipped by the store), or, for one part of a split unit, into
+      // its workspace slot with the rows' running max and sum beside it
+      // (flash_merge_kernel combines the parts)
       uint8_t* stage = sQ + t * TB;
+      const int slot = partial ? tail_u * p.split + part : 0;
       if (have_o) {
         const float inv_l = 1.f / l;
 #pragma unroll
@@ -775,36 +783,23 @@ __global__ void __launch_bounds__(kFlashThreads, 1) flash_fwd_kernel(const __gri
                 make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
-        if (valid && hf == 0 && p.lse != nullptr)
+        if (partial) {
+          if (hf == 0) p.ws_ml[static_cast<size_t>(slot) * 256 + t * 128 + row] = make_float2(m_use, l);
+        } else if (valid && hf == 0 && p.lse != nullptr) {
           p.lse[(static_cast<size_t>(b) * p.H + h) * p.n_q + q_row] = (m_use + __log2f(l)) * 0.69314718055994531f;
+        }
       }
       fence_proxy_async_smem();
       named_bar_sync(10 + t, 256);  // the tile's eight softmax warps
       if (quarter == 0 && hf == 0 && lane == 0 && !abort_flag && q_base + t * 128 < p.n_q) {
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_store_4d(&p.o_map[c], stage + C::chunk_off(c), 64 * c, h, q_base + t * 128, b);
+        for (int c = 0; c < C::kChunks; ++c) {
+          if (partial)
+            tma_store_4d(&p.ws_map[c], stage + C::chunk_off(c), 64 * c, 0, slot * 256 + t * 128, 0);
+          else
+            tma_store_4d(&p.o_map[c], stage + C::chunk_off(c), 64 * c, h, q_base + t * 128, b);
+        }
         bulk_commit_group();
         bulk_wait_read_all();
-      }
-    }
-    if (partial) {
-      // one part of a split unit: store the unnormalised O row with its
-      // running max and sum (flash_merge_kernel combines the parts)
-      const size_t slot0 = static_cast<size_t>(tail_u) * p.split * 256 + t * 128 + row;
-      if (have_o) {
-        float* po = p.ws_o + (slot0 + static_cast<size_t>(part) * 256) * D + DH * hf;
-#pragma unroll
-        for (int c = 0; c < DH / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(tO + 16 * c, o);
-          tmem_ld_wait16(o);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            reinterpret_cast<float4*>(po + 16 * c)[v] =
-                make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]), __uint_as_float(o[4 * v + 2]),
-                            __uint_as_float(o[4 * v + 3]));
-        }
-        if (hf == 0) p.ws_ml[slot0 + static_cast<size_t>(part) * 256] = make_float2(m_use, l);
       }
     }
   }

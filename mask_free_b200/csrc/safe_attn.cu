@@ -179,8 +179,8 @@ FlashPlan plan_flash(int B, int H, int n_q, int N, int d, int sms) {
   }
   if (pl.split > 1) {
     const size_t slots = static_cast<size_t>(pl.tail) * pl.split * 256;
-    pl.ws_o = 0;
-    pl.ws_ml = align256(slots * d * sizeof(float));
+    pl.ws_o = 0;  // bf16 O / l of the parts
+    pl.ws_ml = align256(slots * d * 2);
     pl.ws_bytes = pl.ws_ml + align256(slots * sizeof(float2));
   }
   return pl;
@@ -197,7 +197,7 @@ safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t
   if (attr_err != cudaSuccess) return SAFE_ERR_CUDA;
   FlashPlan pl = plan_flash(p.B, p.H, p.n_q, p.N, D, device_sms());
   if (pl.split > kMaxSplit) return SAFE_ERR_UNSUPPORTED;  // the merge takes at most kMaxSplit parts
-  if (pl.split > 1 && (ws == nullptr || ws_bytes < pl.ws_bytes)) {
+  if (pl.split > 1 && (!aligned16(ws) || ws_bytes < pl.ws_bytes)) {
     pl.full = pl.units;  // no workspace: whole units only
     pl.split = 1;
     pl.tail = 0;
@@ -205,12 +205,14 @@ safe_status launch_flash(FlashParams& p, void* ws, size_t ws_bytes, cudaStream_t
   p.n_mblk = (p.n_q + 255) / 256;
   p.full_units = pl.full;
   p.split = pl.split;
-  p.ws_o = nullptr;
+  p.ws_ob = nullptr;
   p.ws_ml = nullptr;
   if (pl.split > 1) {
     uint8_t* w = static_cast<uint8_t*>(ws);
-    p.ws_o = reinterpret_cast<float*>(w + pl.ws_o);
+    p.ws_ob = reinterpret_cast<__nv_bfloat16*>(w + pl.ws_o);
     p.ws_ml = reinterpret_cast<float2*>(w + pl.ws_ml);
+    for (int c = 0; c < nchunks(D); ++c)
+      if (!encode_rows_map(&p.ws_map[c], p.ws_ob, 1, pl.tail * pl.split * 256, 1, D, c)) return SAFE_ERR_CUDA;
   }
   const unsigned grid = static_cast<unsigned>(pl.full + pl.tail * pl.split);
   // both launches are programmatic dependents of what precedes them in the
