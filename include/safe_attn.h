@@ -103,9 +103,11 @@ safe_status safe_mask_classify_sync(const void* mask, int dtype, const int64_t s
  *           bytes (256-byte aligned), or NULL. With it, the units of the
  *           last, partial wave of CTAs are split into key ranges whose
  *           partial results a second small kernel merges (balances the
- *           wave); without it every CTA takes all keys. Either way the
- *           result is the same up to fp32 rounding order. Contents need no
- *           initialisation; the size is 0 when no split pays off.
+ *           wave); without it every CTA takes all keys. The parts keep
+ *           their O / l in bf16 beside their fp32 running max and sum, so a
+ *           split row carries one more bf16 rounding (2^-9 relative) than
+ *           an unsplit one. Contents need no initialisation; the size is 0
+ *           when no split pays off.
  * fp32 accumulation and softmax; O is rounded to bf16 (nearest even).
  */
 size_t safe_attn_workspace_bytes(int B, int n_q, int N, int H, int d);
