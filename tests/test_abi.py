@@ -67,6 +67,11 @@ def test_attn_workspace_plan(lib):
     assert lib.safe_srsu_workspace_bytes(1, 64, 256, 2, 80) == 0
     assert lib.safe_attn_workspace_bytes(0, 256, 256, 2, 64) == 0
     assert lib.safe_attn_workspace_bytes(1, 256, 256, 2, 80) == 0
+    # dense N = 4096 on 148 SMs: 768 units, the last 28 split into 4 key
+    # parts; a part keeps 256 rows of bf16 O / l and 256 (m, l) pairs
+    slots = 28 * 4 * 256
+    assert lib.safe_attn_workspace_bytes(2, 4096, 4096, 24, 96) == \
+        -(-slots * 96 * 2 // 256) * 256 + -(-slots * 8 // 256) * 256
 
 
 def test_workspace_size(lib):
