@@ -6,7 +6,13 @@
 //     Y[b, r, :] = act( X[b, S[b, r], :] W^T + bias )
 // (no S: every row in order, the dense block of Eq. (18)).
 //
-// Persistent kernel: one CTA per SM walks the 128 x 256 output tiles
+// Two kernels share the epilogue below: linear_pair_kernel (CTA pairs,
+// 256 x 256 tiles; every row in order, which the entry point also uses for
+// the rows of S once it has copied them into a compact matrix) and
+// linear_kernel (one SM per 128 x 256 tile; it gathers the rows of S
+// itself when there is no workspace for the copy).
+//
+// linear_kernel is persistent: one CTA per SM walks the 128 x 256 output tiles
 // t = blockIdx.x, blockIdx.x + gridDim.x, ... (the column tile fastest, so
 // CTAs running at the same time share their gathered rows of X through L2).
 //   warp 0     producer: per 64-wide K chunk, the 128 rows of X (rows of
